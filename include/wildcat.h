@@ -1,0 +1,153 @@
+/*
+ * wildcat.h — C ABI of the B200 (sm_100a) WildCat coreset-attention library.
+ *
+ * WildCat approximates softmax attention by attending over a small weighted
+ * coreset of the keys:
+ *   1. select   randomly pivoted Cholesky (RPCholesky) on the exponential
+ *               kernel H = exp(beta K K^T) picks r pivot keys S and the
+ *               partial Cholesky factor F (n x r, F F^T ~ H).
+ *               [WildCat: Near-Linear Attention in Theory and Practice,
+ *                gist.science technical summary, "Methodik" item 1]
+ *   2. weights  Nystrom weights on [V | 1]:
+ *               W = h(K_S,K_S)^+ h(K_S,K) [V | 1]     (r x (dv+1))
+ *               [same page, "Methodik" item 2: W = h(K_S,K_S)^+ h(K_S,K),
+ *                compressed values V_S = W V; the extra column carries the
+ *                softmax normaliser]
+ *   3. attend   out = rownorm(exp(beta Q K_S^T) W): the last column of the
+ *               product divides the others.
+ *               [same title, gptget.net page, Abstract: attend over only a
+ *                small weighted coreset]
+ * h(x, y) = exp(beta <x, y>), beta = 1/sqrt(d) unless `scale` says otherwise.
+ *
+ * Conventions shared by every call
+ *   - Pointers are DEVICE pointers owned by the caller; the library allocates
+ *     no device memory.  Scratch lives in the caller's workspace `ws` of at
+ *     least wc_workspace_bytes(shape) bytes, 256-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on it; argument errors are returned before any
+ *     launch, launch errors as WC_ERR_CUDA.  Errors that a kernel meets on
+ *     the device (a wait that ran out, a non-finite factor) are recorded in
+ *     the workspace and reported by wc_check_device_status.
+ *   - Tensors are dense, row-major, 16-byte aligned:
+ *       Q   [B, Hq,  n_q, d]    dtype
+ *       K   [B, Hkv, n_k, d]    dtype
+ *       V   [B, Hkv, n_k, dv]   dtype
+ *       piv [B, Hkv, r]         int32, pivot key indices in draw order;
+ *                               entries >= rank are -1
+ *       rank[B, Hkv]            int32, pivots accepted (<= r)
+ *       F   [B, Hkv, r, ldf]    fp32, ldf = wc_f_ld(n_k); F[.., c, i] is the
+ *                               factor entry of key i in column c; columns
+ *                               >= rank and entries i >= n_k are zero
+ *       Ks  [B, Hkv, r, d]      dtype, the pivot keys K[piv]; rows >= rank zero
+ *       W   [B, Hkv, r, dv+1]   fp32; rows >= rank zero
+ *       out [B, Hq,  n_q, dv]   fp32
+ *     Query head g reads kv head g / (Hq / Hkv) (grouped-query attention).
+ *   - Results are deterministic for a given shape, seed and GPU.
+ */
+#ifndef WILDCAT_H
+#define WILDCAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WC_OK = 0,
+    WC_ERR_INVALID = 1,      /* bad shape, null or misaligned pointer */
+    WC_ERR_CUDA = 2,         /* a CUDA runtime call or launch failed */
+    WC_ERR_TIMEOUT = 3,      /* a device-side wait ran out (recorded on the device) */
+    WC_ERR_UNSUPPORTED = 4,  /* valid but not implemented (e.g. d not in {64, 128} on a path) */
+    WC_ERR_WORKSPACE = 5,    /* ws_bytes < wc_workspace_bytes(shape) */
+    WC_ERR_NUMERIC = 6       /* non-finite value met on the device */
+} wc_status;
+
+typedef enum { WC_F32 = 0, WC_BF16 = 1 } wc_dtype;
+
+typedef struct {
+    int32_t batch;    /* B >= 1 */
+    int32_t hq;       /* query heads, a multiple of hkv */
+    int32_t hkv;      /* key/value heads >= 1 */
+    int32_t n_k;      /* keys per head, 1 <= n_k <= 2^26 */
+    int32_t n_q;      /* queries per head >= 0 */
+    int32_t d;        /* key/query width, a multiple of 8, 8..256 */
+    int32_t dv;       /* value width, a multiple of 8, 8..256 */
+    int32_t r;        /* coreset size requested, 1 <= r <= min(n_k, 4096) */
+    int32_t dtype;    /* wc_dtype of Q, K, V and Ks */
+    float scale;      /* beta; 0 selects 1/sqrt(d) */
+    float eps_stop;   /* stop rule: selection ends when the drawn pivot's residual
+                         is <= eps_stop * max_i H_ii; 0 selects 2^-20 */
+    uint32_t wait_timeout_ms;  /* bound on every device-side wait; 0 selects 10000 */
+    uint64_t seed;    /* Philox4x32-10 key of the pivot draws */
+} wc_shape;
+
+/* Row stride (elements) of F for n_k keys: n_k rounded up to a multiple of 8. */
+int64_t wc_f_ld(int32_t n_k);
+
+/* Workspace bytes the calls below need for `shape` (0 if the shape is invalid). */
+size_t wc_workspace_bytes(const wc_shape* shape);
+
+/*
+ * select — RPCholesky [Methodik item 1].  For each (b, kv head) unit u = b*Hkv+h:
+ *   d_i = H_ii = exp(beta |k_i|^2);   for j = 0 .. r-1:
+ *     u_j = Philox4x32-10(ctr = (j, u, 0, 0), key = seed).x0 * 2^-32
+ *     s_j = smallest i with d_0 + ... + d_i > u_j * sum(d)  (inverse CDF)
+ *     stop (rank = j) if sum(d) <= 0 or d_{s_j} <= eps_stop * max_i H_ii
+ *     F[:, j] = (H[:, s_j] - F[:, :j] F[s_j, :j]^T) / sqrt(d_{s_j}),
+ *               with the entries at earlier pivots set to zero
+ *     d_i = max(d_i - F[i, j]^2, 0);  d_{s_j} = 0
+ * Writes piv, F and rank.
+ */
+wc_status wc_select(const wc_shape* shape, const void* K, int32_t* piv, float* F,
+                    int32_t* rank, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * weights — Nystrom weights [Methodik item 2] from select's outputs:
+ *   Ks = K[piv];  C1 = exp(beta Ks K^T) [V | 1];  L = F[piv, :rank] (lower
+ *   triangular, L L^T = h(K_S, K_S));  W = L^-T (L^-1 C1).
+ * Writes Ks and W.
+ */
+wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const int32_t* piv,
+                     const float* F, const int32_t* rank, void* Ks, float* W,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * attend — coreset attention [Abstract]: A = exp(beta Q Ks^T) W over the
+ * first rank[u] coreset rows;  out[q, c] = A[q, c] / A[q, dv].
+ */
+wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const float* W,
+                    const int32_t* rank, float* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * forward — select, weights and attend back to back on `stream` with no host
+ * synchronisation.  piv, rank, F, Ks and W may be NULL, in which case they
+ * live in the workspace (wc_workspace_bytes counts them).
+ */
+wc_status wc_forward(const wc_shape* shape, const void* Q, const void* K, const void* V,
+                     float* out, int32_t* piv, int32_t* rank, float* F, void* Ks, float* W,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, returns the first error a kernel recorded in `ws`
+ * since the last check (WC_OK if none) and clears the record.
+ */
+wc_status wc_check_device_status(void* ws, void* stream);
+
+/*
+ * Exercises the bounded device-side wait that select uses between the
+ * thread blocks of one unit: two blocks meet at a barrier that one of them
+ * never reaches, so the other gives up after timeout_ms and records
+ * WC_ERR_TIMEOUT in `ws` (read it with wc_check_device_status).  No fault,
+ * no trap; the context stays usable.  ws needs 4096 bytes.
+ */
+wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_ms, void* stream);
+
+/* Static text for a status code. */
+const char* wc_status_string(wc_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
