@@ -1,0 +1,187 @@
+// api.cu — the C ABI (include/wildcat.h): argument checks, workspace layout,
+// and the launch sequences of select, weights, attend and forward.
+#include <math.h>
+#include <string.h>
+
+#include "wc_common.cuh"
+#include "wc_expmm.cuh"
+#include "wc_internal.h"
+
+namespace wc {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static int64_t f_ld(int32_t n) { return ((int64_t)n + 7) / 8 * 8; }
+
+wc_status make_shape(const wc_shape* in, Shape* o) {
+    if (!in) return WC_ERR_INVALID;
+    const wc_shape& s = *in;
+    if (s.batch < 1 || s.hkv < 1 || s.hq < 1 || s.hq % s.hkv != 0) return WC_ERR_INVALID;
+    if (s.n_k < 1 || s.n_k > (1 << 26) || s.n_q < 0) return WC_ERR_INVALID;
+    if (s.d < 8 || s.d > 256 || s.d % 8 || s.dv < 8 || s.dv > 256 || s.dv % 8) return WC_ERR_INVALID;
+    if (s.r < 1 || s.r > s.n_k || s.r > 4096) return WC_ERR_INVALID;
+    if (s.dtype != WC_F32 && s.dtype != WC_BF16) return WC_ERR_INVALID;
+    if (!(s.scale >= 0.f) || !isfinite(s.scale) || !(s.eps_stop >= 0.f) || !isfinite(s.eps_stop))
+        return WC_ERR_INVALID;
+    if ((long long)s.batch * s.hq > 65535) return WC_ERR_INVALID;  // grid z of the attend launch
+    o->batch = s.batch; o->hq = s.hq; o->hkv = s.hkv;
+    o->n = s.n_k; o->nq = s.n_q; o->d = s.d; o->dv = s.dv; o->r = s.r;
+    o->dtype = s.dtype;
+    o->beta = s.scale > 0.f ? (double)s.scale : 1.0 / sqrt((double)s.d);
+    o->eps = s.eps_stop > 0.f ? (double)s.eps_stop : 0x1p-20;
+    o->seed = s.seed;
+    o->timeout_ns = (uint64_t)(s.wait_timeout_ms ? s.wait_timeout_ms : 10000u) * 1000000ull;
+    o->ldf = f_ld(s.n_k);
+    o->units = s.batch * s.hkv;
+    o->esize = s.dtype == WC_BF16 ? 2 : 4;
+    o->nsplit = (s.n_k + kSplitKeys - 1) / kSplitKeys;
+    return WC_OK;
+}
+
+WsLayout make_layout(const Shape& s) {
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, kWsAlign);
+        return at;
+    };
+    const size_t U = (size_t)s.units;
+    L.status = take(256);
+    L.sync = take(sizeof(UnitSync) * U);
+    L.partials = take(sizeof(double) * U * 2 * kMaxBlocksPerUnit);
+    L.kt = take((size_t)s.esize * U * s.d * s.ldf);
+    L.lg = take(sizeof(float) * U * s.r * s.r);
+    L.c1part = take(sizeof(float) * U * s.nsplit * s.r * (s.dv + 2));
+    L.y = take(sizeof(double) * U * s.r * (s.dv + 1));
+    L.scratch_end = off;
+    L.piv = take(sizeof(int32_t) * U * s.r);
+    L.rank = take(sizeof(int32_t) * U);
+    L.f = take(sizeof(float) * U * s.r * s.ldf);
+    L.ks = take((size_t)s.esize * U * s.r * s.d);
+    L.w = take(sizeof(float) * U * s.r * (s.dv + 1));
+    L.forward_end = off;
+    return L;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static wc_status check_ws(const Shape& s, void* ws, size_t ws_bytes, bool forward_room) {
+    if (!ws || ((uintptr_t)ws & (kWsAlign - 1))) return WC_ERR_INVALID;
+    const WsLayout L = make_layout(s);
+    if (ws_bytes < (forward_room ? L.forward_end : L.scratch_end)) return WC_ERR_WORKSPACE;
+    return WC_OK;
+}
+
+}  // namespace wc
+
+using namespace wc;
+
+extern "C" {
+
+int64_t wc_f_ld(int32_t n_k) { return n_k < 1 ? 0 : f_ld(n_k); }
+
+size_t wc_workspace_bytes(const wc_shape* shape) {
+    Shape s;
+    if (make_shape(shape, &s) != WC_OK) return 0;
+    return make_layout(s).scratch_end;
+}
+
+size_t wc_forward_workspace_bytes(const wc_shape* shape) {
+    Shape s;
+    if (make_shape(shape, &s) != WC_OK) return 0;
+    return make_layout(s).forward_end;
+}
+
+wc_status wc_select(const wc_shape* shape, const void* K, int32_t* piv, float* F, int32_t* rank, void* ws,
+                    size_t ws_bytes, void* stream) {
+    Shape s;
+    wc_status e = make_shape(shape, &s);
+    if (e != WC_OK) return e;
+    if (!K || !piv || !F || !rank || !aligned16(K) || !aligned16(F) || !aligned16(piv)) return WC_ERR_INVALID;
+    if ((e = check_ws(s, ws, ws_bytes, false)) != WC_OK) return e;
+    return launch_select(s, K, piv, F, rank, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const int32_t* piv, const float* F,
+                     const int32_t* rank, void* Ks, float* W, void* ws, size_t ws_bytes, void* stream) {
+    Shape s;
+    wc_status e = make_shape(shape, &s);
+    if (e != WC_OK) return e;
+    if (!K || !V || !piv || !F || !rank || !Ks || !W) return WC_ERR_INVALID;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(F) || !aligned16(Ks) || !aligned16(W)) return WC_ERR_INVALID;
+    if ((e = check_ws(s, ws, ws_bytes, false)) != WC_OK) return e;
+    char* w = static_cast<char*>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((e = launch_gather(s, K, piv, F, rank, Ks, w, st)) != WC_OK) return e;
+    if ((e = launch_coreset_values(s, Ks, K, V, rank, w, st)) != WC_OK) return e;
+    return launch_solve(s, rank, W, w, st);
+}
+
+wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const float* W, const int32_t* rank,
+                    float* out, void* ws, size_t ws_bytes, void* stream) {
+    Shape s;
+    wc_status e = make_shape(shape, &s);
+    if (e != WC_OK) return e;
+    if (s.nq == 0) return WC_OK;
+    if (!Q || !Ks || !W || !rank || !out) return WC_ERR_INVALID;
+    if (!aligned16(Q) || !aligned16(Ks) || !aligned16(W) || !aligned16(out)) return WC_ERR_INVALID;
+    if ((e = check_ws(s, ws, ws_bytes, false)) != WC_OK) return e;
+    return launch_attend(s, Q, Ks, W, rank, out, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+wc_status wc_forward(const wc_shape* shape, const void* Q, const void* K, const void* V, float* out, int32_t* piv,
+                     int32_t* rank, float* F, void* Ks, float* W, void* ws, size_t ws_bytes, void* stream) {
+    Shape s;
+    wc_status e = make_shape(shape, &s);
+    if (e != WC_OK) return e;
+    if (!K || !V || (s.nq > 0 && (!Q || !out))) return WC_ERR_INVALID;
+    const bool room = !piv || !rank || !F || !Ks || !W;
+    if ((e = check_ws(s, ws, ws_bytes, room)) != WC_OK) return e;
+    const WsLayout L = make_layout(s);
+    char* w = static_cast<char*>(ws);
+    if (!piv) piv = reinterpret_cast<int32_t*>(w + L.piv);
+    if (!rank) rank = reinterpret_cast<int32_t*>(w + L.rank);
+    if (!F) F = reinterpret_cast<float*>(w + L.f);
+    if (!Ks) Ks = w + L.ks;
+    if (!W) W = reinterpret_cast<float*>(w + L.w);
+    if ((e = wc_select(shape, K, piv, F, rank, ws, ws_bytes, stream)) != WC_OK) return e;
+    if ((e = wc_weights(shape, K, V, piv, F, rank, Ks, W, ws, ws_bytes, stream)) != WC_OK) return e;
+    if (s.nq == 0) return WC_OK;
+    return wc_attend(shape, Q, Ks, W, rank, out, ws, ws_bytes, stream);
+}
+
+wc_status wc_check_device_status(void* ws, void* stream) {
+    if (!ws) return WC_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return WC_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return WC_ERR_CUDA;
+    if (host != 0) {
+        if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return WC_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return static_cast<wc_status>(host);
+}
+
+wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_ms, void* stream) {
+    if (!ws || ws_bytes < 4096 || ((uintptr_t)ws & (kWsAlign - 1))) return WC_ERR_INVALID;
+    if (timeout_ms == 0 || timeout_ms > 60000) return WC_ERR_INVALID;
+    return launch_wait_selftest(static_cast<char*>(ws), (uint64_t)timeout_ms * 1000000ull,
+                                static_cast<cudaStream_t>(stream));
+}
+
+const char* wc_status_string(wc_status status) {
+    switch (status) {
+        case WC_OK: return "ok";
+        case WC_ERR_INVALID: return "invalid argument";
+        case WC_ERR_CUDA: return "CUDA error";
+        case WC_ERR_TIMEOUT: return "device-side wait timed out";
+        case WC_ERR_UNSUPPORTED: return "unsupported shape";
+        case WC_ERR_WORKSPACE: return "workspace too small";
+        case WC_ERR_NUMERIC: return "non-finite value on the device";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,521 @@
+// select.cu — randomly pivoted Cholesky on H = exp(beta K K^T), one persistent
+// launch per wave of units.
+//
+// Method: WildCat: Near-Linear Attention in Theory and Practice (gist.science
+// technical summary, "Methodik" item 1): a partial Cholesky factorisation of
+// the exponential kernel matrix whose pivot at every step is drawn from the
+// diagonal of the current residual matrix.
+//
+// Design (B200): each (batch, kv-head) unit owns C thread blocks; block c owns
+// a contiguous slice of rows (keys).  The residual diagonal of the slice stays
+// in shared memory in fp64 for the whole run.  A step is
+//   1. every block reads the C slice sums of the residual diagonal (fp64,
+//      written at the end of the previous step), draws t = u_j * sum with
+//      Philox4x32-10 and finds the block whose slice holds the crossing;
+//   2. that block scans its slice (inverse CDF, strict ">") and publishes the
+//      pivot s_j and its residual through the unit's sync slot;
+//   3. every block streams, for its rows i, the transposed keys Kt[:, i] and
+//      the factor columns F[0..j), i (both laid out with i contiguous, so a
+//      warp reads 512 contiguous bytes per column) and computes
+//        F[j, i] = (exp(beta <k_i, k_s>) - sum_c F[c, i] F[c, s]) / sqrt(d_s)
+//      with fp32 products summed in chunks of eight into fp64, then downdates
+//      its residual diagonal and publishes its new slice sum;
+//   4. a bounded barrier among the unit's blocks closes the step.
+// Blocks of one unit wait on each other, so a wave with C > 1 is launched
+// cooperatively (all blocks co-resident); every wait gives up after the
+// shape's timeout and records WC_ERR_TIMEOUT.
+#include "wc_common.cuh"
+#include "wc_internal.h"
+
+namespace wc {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kGroup = 8;  // rows per thread per pass (two float4 of F)
+
+struct SelectArgs {
+    const void* K;
+    int32_t* piv;
+    float* F;
+    int32_t* rank;
+    void* Kt;
+    UnitSync* sync;
+    double* partials;
+    int* status;
+    int64_t ldf;
+    int32_t n, d, r;
+    int32_t C;      // blocks per unit
+    int32_t m;      // rows per block (multiple of kGroup)
+    int32_t unit0;  // first unit of this wave
+    double beta, eps;
+    uint64_t seed;
+    uint64_t timeout_ns;
+};
+
+// Shared-memory plan (bytes) for m rows, r pivots, d dims.
+__host__ __device__ inline size_t select_smem_bytes(int m, int r, int d) {
+    return (size_t)m * 8          // residual diagonal (fp64)
+           + (size_t)kThreads * 8 // per-thread inclusive scan
+           + (size_t)d * 8        // pivot key
+           + (size_t)r * 4        // F[s, 0..j)
+           + (size_t)m            // pivot flags
+           + 64;                  // broadcast scalars
+}
+
+struct Bcast {
+    double base, tau, d_s;
+    int owner, stop, s, ok, tstar, pad;
+};
+
+// Inclusive scan over the block of one double per thread (fixed order,
+// deterministic); writes each thread's inclusive value to scan[tid] and
+// returns the block total.
+__device__ double block_scan(double v, double* scan) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    __shared__ double wtot[kThreads / 32];
+    if (lane == 31) wtot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        double w = lane < kThreads / 32 ? wtot[lane] : 0.0;
+#pragma unroll
+        for (int o = 1; o < kThreads / 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < kThreads / 32) wtot[lane] = w;
+    }
+    __syncthreads();
+    if (warp > 0) v += wtot[warp - 1];
+    scan[threadIdx.x] = v;
+    const double total = wtot[kThreads / 32 - 1];
+    __syncthreads();
+    return total;
+}
+
+// Contiguous chunk of the slice that thread `t` sums for the scans.
+__device__ __forceinline__ void chunk_of(int t, int mlen, int* lo, int* hi) {
+    const int q = (mlen + kThreads - 1) / kThreads;
+    *lo = min(mlen, t * q);
+    *hi = min(mlen, *lo + q);
+}
+
+__device__ __forceinline__ void unpack_bf16x8(uint4 raw, float x[8]) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        x[2 * k] = __uint_as_float(w[k] << 16);
+        x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+}
+
+// <k_i, k_s> for the 8 rows at Kt + i0 (column stride ldf).
+template <typename T>
+__device__ __forceinline__ void key_dots(const T* Kt, int64_t ldf, int d, const double* ks, double dot[8]);
+
+template <>
+__device__ __forceinline__ void key_dots<__nv_bfloat16>(const __nv_bfloat16* Kt, int64_t ldf, int d,
+                                                       const double* ks, double dot[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dot[k] = 0.0;
+    for (int c0 = 0; c0 < d; c0 += 8) {
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            float x[8];
+            unpack_bf16x8(ld_stream_u4(Kt + (int64_t)(c0 + c) * ldf), x);
+            const float kc = (float)ks[c0 + c];  // exact: ks holds bf16 values
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fmaf(x[k], kc, acc[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dot[k] += (double)acc[k];
+    }
+}
+
+template <>
+__device__ __forceinline__ void key_dots<float>(const float* Kt, int64_t ldf, int d, const double* ks,
+                                               double dot[8]) {
+    // fp32 inputs: products and sums in fp64
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dot[k] = 0.0;
+    for (int c = 0; c < d; ++c) {
+        const float4 a = ld_stream_f4(Kt + (int64_t)c * ldf);
+        const float4 b = ld_stream_f4(Kt + (int64_t)c * ldf + 4);
+        const double kc = ks[c];
+        dot[0] += (double)a.x * kc; dot[1] += (double)a.y * kc;
+        dot[2] += (double)a.z * kc; dot[3] += (double)a.w * kc;
+        dot[4] += (double)b.x * kc; dot[5] += (double)b.y * kc;
+        dot[6] += (double)b.z * kc; dot[7] += (double)b.w * kc;
+    }
+}
+
+// sum_{c<j} F[c, i] F[c, s] for the 8 rows at Fi (column stride ldf).
+__device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, const float* fs,
+                                           double cor[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cor[k] = 0.0;
+    int c0 = 0;
+    for (; c0 + 8 <= j; c0 += 8) {
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float* p = Fi + (int64_t)(c0 + c) * ldf;
+            const float4 a = ld_stream_f4(p), b = ld_stream_f4(p + 4);
+            const float f = fs[c0 + c];
+            acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
+            acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
+            acc[4] = fmaf(b.x, f, acc[4]); acc[5] = fmaf(b.y, f, acc[5]);
+            acc[6] = fmaf(b.z, f, acc[6]); acc[7] = fmaf(b.w, f, acc[7]);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cor[k] += (double)acc[k];
+    }
+    if (c0 < j) {
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        for (int c = c0; c < j; ++c) {
+            const float* p = Fi + (int64_t)c * ldf;
+            const float4 a = ld_stream_f4(p), b = ld_stream_f4(p + 4);
+            const float f = fs[c];
+            acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
+            acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
+            acc[4] = fmaf(b.x, f, acc[4]); acc[5] = fmaf(b.y, f, acc[5]);
+            acc[6] = fmaf(b.z, f, acc[6]); acc[7] = fmaf(b.w, f, acc[7]);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cor[k] += (double)acc[k];
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int tid = threadIdx.x;
+    const int unit = a.unit0 + blockIdx.x / a.C;
+    const int blk = blockIdx.x % a.C;
+    const int n = a.n, d = a.d, r = a.r;
+    const int64_t ldf = a.ldf;
+    const int r0 = min(n, blk * a.m);
+    const int r1 = min(n, r0 + a.m);
+    const int mlen = r1 - r0;
+    const int ng = (mlen + kGroup - 1) / kGroup;
+
+    double* dg = reinterpret_cast<double*>(smem);
+    double* scan = dg + a.m;
+    double* ks = scan + kThreads;
+    float* fs = reinterpret_cast<float*>(ks + d);
+    unsigned char* ispiv = reinterpret_cast<unsigned char*>(fs + r);
+    __shared__ Bcast bc;
+
+    const T* K = static_cast<const T*>(a.K) + (size_t)unit * n * d;
+    T* Kt = static_cast<T*>(a.Kt) + (size_t)unit * d * ldf;
+    float* F = a.F + (size_t)unit * r * ldf;
+    UnitSync* us = a.sync + unit;
+    double* part = a.partials + (size_t)unit * 2 * kMaxBlocksPerUnit;
+    int* status = a.status;
+
+    // ---- initial residual: d_i = H_ii = exp(beta |k_i|^2); transpose the slice
+    double lmax = 0.0;
+    for (int il = tid; il < ng * kGroup; il += kThreads) {
+        const int i = r0 + il;
+        if (il < mlen) {
+            const T* krow = K + (size_t)i * d;
+            double ss = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const T v = krow[c];
+                const double x = (double)to_f32(v);
+                ss += x * x;
+                Kt[(int64_t)c * ldf + i] = v;
+            }
+            dg[il] = exp(a.beta * ss);
+            lmax = fmax(lmax, dg[il]);
+        } else {
+            for (int c = 0; c < d; ++c) Kt[(int64_t)c * ldf + i] = T(0.f);
+            dg[il] = 0.0;
+        }
+        ispiv[il] = 0;
+    }
+    // block max of H_ii -> unit max (positive doubles order like their bits)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if ((tid & 31) == 0 && lmax > 0.0) atomicMax(&us->hmax_bits, (unsigned long long)__double_as_longlong(lmax));
+
+    {
+        int lo, hi;
+        chunk_of(tid, mlen, &lo, &hi);
+        double sum = 0.0;
+        for (int il = lo; il < hi; ++il) sum += dg[il];
+        const double tot = block_scan(sum, scan);
+        if (tid == 0) part[blk] = tot;
+    }
+    bool alive = unit_barrier(&us->bar, a.C, 1, a.timeout_ns, status, &bc.ok);
+    double hmax = 0.0;
+    if (alive) {
+        hmax = __longlong_as_double((long long)__ldcg(&us->hmax_bits));
+        if (!isfinite(hmax)) {
+            if (tid == 0) record_status(status, WC_ERR_NUMERIC);
+            alive = false;
+        }
+    }
+
+    int final_rank = alive ? r : 0;
+    for (int j = 0; alive && j < r; ++j) {
+        const double* pj = part + (size_t)(j & 1) * kMaxBlocksPerUnit;
+        // 1. which block's slice holds t = u_j * sum(d)
+        if (tid == 0) {
+            double total = 0.0;
+            for (int c = 0; c < a.C; ++c) total += __ldcg(pj + c);
+            bc.stop = 0;
+            bc.owner = -1;
+            if (!(total > 0.0)) {
+                if (isnan(total)) record_status(status, WC_ERR_NUMERIC);
+                bc.stop = 1;
+            } else {
+                const double tau = pivot_uniform(a.seed, (uint32_t)j, (uint32_t)unit) * total;
+                double run = 0.0;
+                for (int c = 0; c < a.C; ++c) {
+                    const double nxt = run + __ldcg(pj + c);
+                    if (nxt > tau) { bc.owner = c; bc.base = run; break; }
+                    run = nxt;
+                }
+                if (bc.owner < 0) {  // rounding left tau at the top: last block with mass
+                    run = 0.0;
+                    for (int c = 0; c < a.C; ++c) {
+                        const double p = __ldcg(pj + c);
+                        if (p > 0.0) { bc.owner = c; bc.base = run; }
+                        run += p;
+                    }
+                }
+                bc.tau = tau;
+            }
+            bc.tstar = kThreads;
+        }
+        __syncthreads();
+        if (bc.stop) { final_rank = j; break; }
+
+        // 2. the owner block finds the pivot in its slice and publishes it
+        if (blk == bc.owner) {
+            const double base = bc.base, tau = bc.tau;
+            if (base + scan[tid] > tau) atomicMin(&bc.tstar, tid);
+            __syncthreads();
+            if (tid == 0 && bc.tstar == kThreads) bc.tstar = kThreads - 1;  // rounding guard
+            __syncthreads();
+            if (tid == bc.tstar) {
+                int lo, hi;
+                chunk_of(tid, mlen, &lo, &hi);
+                double run = tid == 0 ? base : base + scan[tid - 1];
+                int sl = -1;
+                for (int il = lo; il < hi; ++il) {
+                    run += dg[il];
+                    if (run > tau) { sl = il; break; }
+                }
+                if (sl < 0) {  // rounding: last positive entry of the chunk, else of the slice
+                    for (int il = hi - 1; il >= lo && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                    for (int il = mlen - 1; il >= 0 && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                }
+                const double ds = sl >= 0 ? dg[sl] : 0.0;
+                const int stop = !(ds > a.eps * hmax);
+                us->s = r0 + sl;
+                us->d_s = ds;
+                us->stop = stop;
+                if (!stop) a.piv[(size_t)unit * r + j] = r0 + sl;
+                __threadfence();
+                st_release_u32(&us->pivflag, (uint32_t)j + 1u);
+                bc.s = r0 + sl;
+                bc.d_s = ds;
+                bc.stop = stop;
+            }
+            __syncthreads();
+        } else {
+            if (tid == 0) {
+                if (wait_geq(&us->pivflag, (uint32_t)j + 1u, a.timeout_ns, status)) {
+                    bc.s = *(volatile int32_t*)&us->s;
+                    bc.d_s = *(volatile double*)&us->d_s;
+                    bc.stop = *(volatile int32_t*)&us->stop;
+                    bc.ok = 1;
+                } else {
+                    bc.ok = 0;
+                }
+            }
+            __syncthreads();
+            if (!bc.ok) { final_rank = j; alive = false; break; }
+        }
+        if (bc.stop) { final_rank = j; break; }
+        const int s = bc.s;
+        const double ds = bc.d_s;
+
+        // 3. pivot key and F[s, 0..j) into shared memory
+        for (int c = tid; c < d; c += kThreads) ks[c] = (double)to_f32(K[(size_t)s * d + c]);
+        for (int c = tid; c < j; c += kThreads) fs[c] = ld_cg_f32(F + (int64_t)c * ldf + s);
+        __syncthreads();
+
+        // 4. column j over this block's rows, and the residual downdate
+        const double root = sqrt(ds);
+        float* Fj = F + (int64_t)j * ldf;
+        for (int g = tid; g < ng; g += kThreads) {
+            const int il0 = g * kGroup;
+            const int i0 = r0 + il0;
+            double dot[8], cor[8];
+            key_dots<T>(Kt + i0, ldf, d, ks, dot);
+            correction(F + i0, ldf, j, fs, cor);
+            float out[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int il = il0 + k;
+                double f = 0.0;
+                if (il < mlen && !ispiv[il]) f = (exp(a.beta * dot[k]) - cor[k]) / root;
+                out[k] = (float)f;
+                if (il < mlen) {
+                    const double nd = dg[il] - f * f;
+                    dg[il] = nd > 0.0 ? nd : 0.0;
+                }
+            }
+            *reinterpret_cast<float4*>(Fj + i0) = make_float4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<float4*>(Fj + i0 + 4) = make_float4(out[4], out[5], out[6], out[7]);
+        }
+        __syncthreads();
+        if (s >= r0 && s < r1 && tid == 0) {
+            dg[s - r0] = 0.0;
+            ispiv[s - r0] = 1;
+        }
+        __syncthreads();
+
+        // 5. new slice sum, then close the step
+        {
+            int lo, hi;
+            chunk_of(tid, mlen, &lo, &hi);
+            double sum = 0.0;
+            for (int il = lo; il < hi; ++il) sum += dg[il];
+            const double tot = block_scan(sum, scan);
+            if (tid == 0) part[(size_t)((j + 1) & 1) * kMaxBlocksPerUnit + blk] = tot;
+        }
+        if (!unit_barrier(&us->bar, a.C, (uint32_t)j + 2u, a.timeout_ns, status, &bc.ok)) {
+            final_rank = j + 1;
+            alive = false;
+            break;
+        }
+    }
+
+    // ---- columns >= rank are zero; piv beyond rank is -1
+    for (int jj = final_rank; jj < r; ++jj) {
+        float* Fj = F + (int64_t)jj * ldf;
+        for (int g = tid; g < ng; g += kThreads) {
+            const int i0 = r0 + g * kGroup;
+            *reinterpret_cast<float4*>(Fj + i0) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(Fj + i0 + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    if (blk == 0) {
+        for (int jj = final_rank + tid; jj < r; jj += kThreads) a.piv[(size_t)unit * r + jj] = -1;
+        if (tid == 0) a.rank[unit] = final_rank;
+    }
+}
+
+template <typename T>
+wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank, char* ws,
+                          cudaStream_t st) {
+    const WsLayout L = make_layout(s);
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WC_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return WC_ERR_CUDA;
+    int max_smem = 0;
+    cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+
+    // rows per block bounded by shared memory (fp64 diagonal + flags)
+    const size_t fixed = select_smem_bytes(0, s.r, s.d) + 1024;
+    if ((size_t)max_smem <= fixed) return WC_ERR_UNSUPPORTED;
+    int m_max = (int)(((size_t)max_smem - fixed) / 9) / kGroup * kGroup;
+    m_max = m_max > (1 << 20) ? (1 << 20) : m_max;
+
+    auto kern = rpcholesky_kernel<T>;
+    // occupancy at the largest slice we might use
+    const int c_min = (s.n + m_max - 1) / m_max;
+    int C = c_min;
+    int m = ((s.n + C - 1) / C + kGroup - 1) / kGroup * kGroup;
+    size_t smem = select_smem_bytes(m, s.r, s.d);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return WC_ERR_CUDA;
+    int bps = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, kThreads, smem) != cudaSuccess || bps < 1)
+        return WC_ERR_CUDA;
+    const long cap = (long)nsm * bps;
+
+    if ((long)s.units * C <= cap) {
+        // spread each unit over more blocks, keeping >= 256 rows per block
+        long want = cap / s.units;
+        const long rows_cap = (s.n + 255) / 256;
+        if (want > rows_cap) want = rows_cap;
+        if (want > kMaxBlocksPerUnit) want = kMaxBlocksPerUnit;
+        if (want > C) C = (int)want;
+        m = ((s.n + C - 1) / C + kGroup - 1) / kGroup * kGroup;
+        C = (s.n + m - 1) / m;
+        smem = select_smem_bytes(m, s.r, s.d);
+    }
+    if (C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
+
+    SelectArgs a;
+    a.K = K; a.piv = piv; a.F = F; a.rank = rank;
+    a.Kt = ws + L.kt;
+    a.sync = reinterpret_cast<UnitSync*>(ws + L.sync);
+    a.partials = reinterpret_cast<double*>(ws + L.partials);
+    a.status = reinterpret_cast<int*>(ws + L.status);
+    a.ldf = s.ldf; a.n = s.n; a.d = s.d; a.r = s.r;
+    a.C = C; a.m = m;
+    a.beta = s.beta; a.eps = s.eps; a.seed = s.seed; a.timeout_ns = s.timeout_ns;
+
+    if (cudaMemsetAsync(ws + L.sync, 0, sizeof(UnitSync) * (size_t)s.units, st) != cudaSuccess) return WC_ERR_CUDA;
+
+    if (C == 1) {
+        a.unit0 = 0;
+        kern<<<s.units, kThreads, smem, st>>>(a);
+        return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+    }
+    // blocks of a unit wait on each other: co-resident waves, cooperative launch
+    const int per_wave = (int)(cap / C);
+    if (per_wave < 1) return WC_ERR_UNSUPPORTED;
+    for (int u0 = 0; u0 < s.units; u0 += per_wave) {
+        a.unit0 = u0;
+        const int nu = s.units - u0 < per_wave ? s.units - u0 : per_wave;
+        void* args[] = {&a};
+        if (cudaLaunchCooperativeKernel((const void*)kern, dim3(nu * C), dim3(kThreads), args, smem, st) !=
+            cudaSuccess)
+            return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
+// Two blocks meet at a unit barrier that block 1 never reaches: block 0's
+// bounded wait runs out and records WC_ERR_TIMEOUT.
+__global__ void wait_selftest_kernel(UnitSync* sync, int* status, uint64_t timeout_ns) {
+    __shared__ int ok;
+    if (blockIdx.x == 1) return;
+    unit_barrier(&sync->bar, 2, 1, timeout_ns, status, &ok);
+}
+
+}  // namespace
+
+wc_status launch_select(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank, char* ws,
+                        cudaStream_t st) {
+    if (s.dtype == WC_BF16) return launch_select_t<__nv_bfloat16>(s, K, piv, F, rank, ws, st);
+    return launch_select_t<float>(s, K, piv, F, rank, ws, st);
+}
+
+wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st) {
+    UnitSync* sync = reinterpret_cast<UnitSync*>(ws + 256);
+    int* status = reinterpret_cast<int*>(ws);
+    if (cudaMemsetAsync(sync, 0, sizeof(UnitSync), st) != cudaSuccess) return WC_ERR_CUDA;
+    wait_selftest_kernel<<<2, 32, 0, st>>>(sync, status, timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+}  // namespace wc

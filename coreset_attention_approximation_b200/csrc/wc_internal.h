@@ -1,0 +1,70 @@
+// wc_internal.h — workspace layout and kernel launchers of the WildCat library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/wildcat.h"
+
+namespace wc {
+
+constexpr int kMaxBlocksPerUnit = 512;   // select: thread blocks that share one unit
+constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1
+constexpr int kWsAlign = 256;
+
+// One per unit, in the workspace; zeroed before every select launch.
+struct UnitSync {
+    uint32_t bar;                 // barrier arrivals (monotonic within a launch)
+    uint32_t pivflag;             // j + 1 once the pivot of step j is published
+    int32_t s;                    // published pivot
+    int32_t stop;                 // 1 when the run ends at the published step
+    double d_s;                   // residual diagonal at the published pivot
+    unsigned long long hmax_bits; // max_i H_ii (bits of a positive double)
+    uint32_t pad[8];
+};
+static_assert(sizeof(UnitSync) == 64, "UnitSync is 64 bytes");
+
+// Byte offsets into the workspace (all kWsAlign-aligned).
+struct WsLayout {
+    size_t status;    // int32 first device error
+    size_t sync;      // UnitSync[units]
+    size_t partials;  // double[units][2][kMaxBlocksPerUnit]
+    size_t kt;        // dtype[units][d][ldf]   transposed keys
+    size_t lg;        // float[units][r][r]     gathered L = F[piv, :]
+    size_t c1part;    // float[units][nsplit][r][dv + 2]  (O | l | m)
+    size_t y;         // double[units][r][dv + 1]
+    size_t scratch_end;
+    // room for outputs that wc_forward keeps in the workspace when not given
+    size_t piv, rank, f, ks, w;
+    size_t forward_end;
+};
+
+struct Shape {
+    int32_t batch, hq, hkv, n, nq, d, dv, r;
+    int32_t dtype;         // wc_dtype
+    double beta, eps;
+    uint64_t seed;
+    uint64_t timeout_ns;
+    int64_t ldf;
+    int32_t units;         // batch * hkv
+    int32_t esize;         // bytes per Q/K/V element
+    int32_t nsplit;        // C1 partial sums
+};
+
+wc_status make_shape(const wc_shape* in, Shape* out);
+WsLayout make_layout(const Shape& s);
+
+// Kernel launchers (each returns WC_OK or WC_ERR_CUDA / WC_ERR_UNSUPPORTED).
+wc_status launch_select(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank,
+                        char* ws, cudaStream_t st);
+wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const float* F,
+                        const int32_t* rank, void* Ks, char* ws, cudaStream_t st);
+wc_status launch_coreset_values(const Shape& s, const void* Ks, const void* K, const void* V,
+                                const int32_t* rank, char* ws, cudaStream_t st);
+wc_status launch_solve(const Shape& s, const int32_t* rank, float* W, char* ws, cudaStream_t st);
+wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const float* W,
+                        const int32_t* rank, float* out, char* ws, cudaStream_t st);
+wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st);
+
+}  // namespace wc

@@ -1,0 +1,205 @@
+"""Python binding of the WildCat C ABI (include/wildcat.h).
+
+Argument marshalling only: every step runs in libwildcat.so's CUDA kernels.
+Tensors are torch CUDA tensors (PyTorch supplies device memory and streams);
+the functions raise if the library is missing or a call fails.
+
+    from coreset_attention_approximation_b200 import wildcat
+    res = wildcat.forward(Q, K, V, r=64, seed=0)        # dict with out, piv, rank, F, Ks, W
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libwildcat.so")
+
+WC_F32, WC_BF16 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "CUDA error", 3: "device-side wait timed out",
+          4: "unsupported shape", 5: "workspace too small", 6: "non-finite value on the device"}
+
+
+class WildcatError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({code})")
+        self.code = code
+
+
+class WcShape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32),
+        ("n_k", ctypes.c_int32), ("n_q", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("dv", ctypes.c_int32), ("r", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("eps_stop", ctypes.c_float), ("wait_timeout_ms", ctypes.c_uint32),
+        ("seed", ctypes.c_uint64),
+    ]
+
+
+EXPORTS = [
+    "wc_f_ld", "wc_workspace_bytes", "wc_forward_workspace_bytes", "wc_select", "wc_weights", "wc_attend",
+    "wc_forward", "wc_check_device_status", "wc_selftest_wait_timeout", "wc_status_string",
+]
+
+_lib = None
+
+
+def lib():
+    """Load libwildcat.so (built by `python -m coreset_attention_approximation_b200.build`)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m coreset_attention_approximation_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        sp = ctypes.POINTER(WcShape)
+        L.wc_f_ld.argtypes, L.wc_f_ld.restype = [ctypes.c_int32], ctypes.c_int64
+        L.wc_workspace_bytes.argtypes, L.wc_workspace_bytes.restype = [sp], sz
+        L.wc_forward_workspace_bytes.argtypes, L.wc_forward_workspace_bytes.restype = [sp], sz
+        L.wc_select.argtypes, L.wc_select.restype = [sp, vp, vp, vp, vp, vp, sz, vp], i32
+        L.wc_weights.argtypes, L.wc_weights.restype = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i32
+        L.wc_attend.argtypes, L.wc_attend.restype = [sp, vp, vp, vp, vp, vp, vp, sz, vp], i32
+        L.wc_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.wc_forward.restype = i32
+        L.wc_check_device_status.argtypes, L.wc_check_device_status.restype = [vp, vp], i32
+        L.wc_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
+        L.wc_selftest_wait_timeout.restype = i32
+        L.wc_status_string.argtypes, L.wc_status_string.restype = [i32], ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise WildcatError(code, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_shape(batch, hq, hkv, n_k, n_q, d, dv, r, dtype, scale=0.0, eps_stop=0.0, seed=0,
+               wait_timeout_ms=0) -> WcShape:
+    code = {torch.float32: WC_F32, torch.bfloat16: WC_BF16}.get(dtype, dtype)
+    return WcShape(batch, hq, hkv, n_k, n_q, d, dv, r, code, scale, eps_stop, wait_timeout_ms, seed)
+
+
+def shape_of(Q, K, V, r, **kw) -> WcShape:
+    B, Hkv, n, d = K.shape
+    dv = V.shape[-1]
+    if Q is None:
+        Hq, nq = Hkv, 0
+    else:
+        Hq, nq = Q.shape[1], Q.shape[2]
+    return make_shape(B, Hq, Hkv, n, nq, d, dv, r, K.dtype, **kw)
+
+
+def f_ld(n_k: int) -> int:
+    return int(lib().wc_f_ld(n_k))
+
+
+def workspace_bytes(shape: WcShape) -> int:
+    return int(lib().wc_workspace_bytes(ctypes.byref(shape)))
+
+
+def forward_workspace_bytes(shape: WcShape) -> int:
+    return int(lib().wc_forward_workspace_bytes(ctypes.byref(shape)))
+
+
+def workspace(shape: WcShape, device, forward_room: bool = False) -> torch.Tensor:
+    n = forward_workspace_bytes(shape) if forward_room else workspace_bytes(shape)
+    if n == 0:
+        raise WildcatError(1, "workspace size")
+    # the device status word at offset 0 starts clear
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _outputs(shape: WcShape, device, dtype):
+    B, Hkv, r, n = shape.batch, shape.hkv, shape.r, shape.n_k
+    return dict(
+        piv=torch.empty(B, Hkv, r, dtype=torch.int32, device=device),
+        rank=torch.empty(B, Hkv, dtype=torch.int32, device=device),
+        F=torch.empty(B, Hkv, r, f_ld(n), dtype=torch.float32, device=device),
+        Ks=torch.empty(B, Hkv, r, shape.d, dtype=dtype, device=device),
+        W=torch.empty(B, Hkv, r, shape.dv + 1, dtype=torch.float32, device=device),
+    )
+
+
+def select(K, r, seed=0, *, ws=None, stream=None, **kw):
+    shape = shape_of(None, K, K[..., :8], r, seed=seed, **kw)
+    o = _outputs(shape, K.device, K.dtype)
+    ws = workspace(shape, K.device) if ws is None else ws
+    _check(lib().wc_select(ctypes.byref(shape), _ptr(K), _ptr(o["piv"]), _ptr(o["F"]), _ptr(o["rank"]),
+                           _ptr(ws), ws.numel(), _stream(stream)), "wc_select")
+    return dict(piv=o["piv"], F=o["F"], rank=o["rank"], ws=ws)
+
+
+def weights(K, V, piv, F, rank, r, *, ws=None, stream=None, **kw):
+    shape = shape_of(None, K, V, r, **kw)
+    o = _outputs(shape, K.device, K.dtype)
+    ws = workspace(shape, K.device) if ws is None else ws
+    _check(lib().wc_weights(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(piv), _ptr(F), _ptr(rank),
+                            _ptr(o["Ks"]), _ptr(o["W"]), _ptr(ws), ws.numel(), _stream(stream)), "wc_weights")
+    return dict(Ks=o["Ks"], W=o["W"], ws=ws)
+
+
+def attend(Q, Ks, W, rank, n_k, *, ws=None, stream=None, **kw):
+    B, Hq, nq, d = Q.shape
+    Hkv, r, dv = Ks.shape[1], Ks.shape[2], W.shape[-1] - 1
+    shape = make_shape(B, Hq, Hkv, n_k, nq, d, dv, r, Q.dtype, **kw)
+    out = torch.empty(B, Hq, nq, dv, dtype=torch.float32, device=Q.device)
+    ws = workspace(shape, Q.device) if ws is None else ws
+    _check(lib().wc_attend(ctypes.byref(shape), _ptr(Q), _ptr(Ks), _ptr(W), _ptr(rank), _ptr(out),
+                           _ptr(ws), ws.numel(), _stream(stream)), "wc_attend")
+    return out
+
+
+def forward(Q, K, V, r, seed=0, *, ws=None, stream=None, outputs=None, **kw):
+    """Whole path on the GPU: select -> weights -> attend.
+
+    Q [B,Hq,nq,d], K [B,Hkv,n,d], V [B,Hkv,n,dv] CUDA tensors (bf16 or fp32,
+    contiguous).  `outputs` may hold preallocated tensors (out, piv, rank, F,
+    Ks, W); missing ones are allocated.  Returns the dict of all of them.
+    """
+    shape = shape_of(Q, K, V, r, seed=seed, **kw)
+    o = dict(outputs or {})
+    for k, v in _outputs(shape, K.device, K.dtype).items():
+        o.setdefault(k, v)
+    o.setdefault("out", torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], shape.dv, dtype=torch.float32,
+                                    device=K.device))
+    ws = workspace(shape, K.device) if ws is None else ws
+    _check(lib().wc_forward(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(o["out"]), _ptr(o["piv"]),
+                            _ptr(o["rank"]), _ptr(o["F"]), _ptr(o["Ks"]), _ptr(o["W"]), _ptr(ws), ws.numel(),
+                            _stream(stream)), "wc_forward")
+    o["ws"] = ws
+    return o
+
+
+def forward_host(Q, K, V, r, seed=0, *, device="cuda", ws=None, stream=None, **kw):
+    """Host-buffer entry: copies Q, K, V (pinned CPU tensors) to the device,
+    runs forward, copies `out` back.  Returns the CPU output tensor."""
+    dq = Q.to(device, non_blocking=True)
+    dk = K.to(device, non_blocking=True)
+    dv = V.to(device, non_blocking=True)
+    res = forward(dq, dk, dv, r, seed, ws=ws, stream=stream, **kw)
+    out = torch.empty(res["out"].shape, dtype=torch.float32, pin_memory=True)
+    out.copy_(res["out"], non_blocking=True)
+    torch.cuda.current_stream().synchronize()
+    return out
+
+
+def check_device_status(ws, stream=None) -> int:
+    return int(lib().wc_check_device_status(_ptr(ws), _stream(stream)))
+
+
+def selftest_wait_timeout(ws, timeout_ms, stream=None) -> int:
+    return int(lib().wc_selftest_wait_timeout(_ptr(ws), ws.numel(), timeout_ms, _stream(stream)))

@@ -67,7 +67,7 @@ typedef enum {
 typedef enum { WC_F32 = 0, WC_BF16 = 1 } wc_dtype;
 
 typedef struct {
-    int32_t batch;    /* B >= 1 */
+    int32_t batch;    /* B >= 1, B * hq <= 65535 */
     int32_t hq;       /* query heads, a multiple of hkv */
     int32_t hkv;      /* key/value heads >= 1 */
     int32_t n_k;      /* keys per head, 1 <= n_k <= 2^26 */
@@ -86,8 +86,13 @@ typedef struct {
 /* Row stride (elements) of F for n_k keys: n_k rounded up to a multiple of 8. */
 int64_t wc_f_ld(int32_t n_k);
 
-/* Workspace bytes the calls below need for `shape` (0 if the shape is invalid). */
+/* Workspace bytes that select, weights, attend and forward need for `shape`
+ * when every output pointer is given (0 if the shape is invalid). */
 size_t wc_workspace_bytes(const wc_shape* shape);
+
+/* Workspace bytes for wc_forward when some of piv, rank, F, Ks, W are NULL:
+ * the scratch above plus room for all five (0 if the shape is invalid). */
+size_t wc_forward_workspace_bytes(const wc_shape* shape);
 
 /*
  * select — RPCholesky [Methodik item 1].  For each (b, kv head) unit u = b*Hkv+h:
@@ -123,7 +128,7 @@ wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const 
 /*
  * forward — select, weights and attend back to back on `stream` with no host
  * synchronisation.  piv, rank, F, Ks and W may be NULL, in which case they
- * live in the workspace (wc_workspace_bytes counts them).
+ * live in the workspace, which must then hold wc_forward_workspace_bytes.
  */
 wc_status wc_forward(const wc_shape* shape, const void* Q, const void* K, const void* V,
                      float* out, int32_t* piv, int32_t* rank, float* F, void* Ks, float* W,
