@@ -35,6 +35,7 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->units = s.batch * s.hkv;
     o->esize = s.dtype == WC_BF16 ? 2 : 4;
     o->nsplit = (s.n_k + kSplitKeys - 1) / kSplitKeys;
+    o->r_pad = (s.r + 63) / 64 * 64;
     return WC_OK;
 }
 
@@ -54,6 +55,11 @@ WsLayout make_layout(const Shape& s) {
     L.lg = take(sizeof(float) * U * s.r * s.r);
     L.c1part = take(sizeof(float) * U * s.nsplit * s.r * (s.dv + 2));
     L.y = take(sizeof(double) * U * s.r * (s.dv + 1));
+    const bool tc = s.dtype == WC_BF16;
+    L.v16 = take(tc ? 2 * U * s.n * s.dv : 0);
+    L.w16 = take(tc ? 2 * U * s.r * s.dv : 0);
+    L.sigma = take(tc ? sizeof(float) * U * s.dv : 0);
+    L.wn = take(tc ? sizeof(float) * U * s.r_pad : 0);
     L.scratch_end = off;
     L.piv = take(sizeof(int32_t) * U * s.r);
     L.rank = take(sizeof(int32_t) * U);

@@ -12,7 +12,7 @@ namespace wc {
 
 wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
                         float* out, char* ws, cudaStream_t st) {
-    (void)ws;
+    if (tc_supported(s)) return launch_attend_tc(s, Q, Ks, W, rank, out, ws, st);
     ExpmmArgs e{};
     e.A = Q; e.a_stride = (int64_t)s.nq * s.d; e.a_rows = s.nq;
     e.B = Ks; e.b_stride = (int64_t)s.r * s.d; e.b_rows = s.r;

@@ -1,0 +1,494 @@
+// expmm_tc.cu — tensor-core (tcgen05 / TMEM / TMA) exp-GEMM of WildCat.
+//
+// For a tile of 128 rows a of A (coreset keys for the weights, queries for
+// attention) and the keys b of B in [b_lo, b_hi):
+//   S = A B^T                    bf16 x bf16 -> fp32 in TMEM (tcgen05.mma)
+//   P = 2^(S beta log2(e) - m)   fp16, in the softmax warps (running max m,
+//                                rescaled only when it grows by more than 2^8)
+//   O += P C                     fp16 x fp16 -> fp32 in TMEM (tcgen05.mma)
+//   l += sum_b P w_b             fp32, in the softmax warps
+// C = fp16 values (V, or the weights W scaled per column); w = 1 or the
+// normaliser column W[:, dv].  Weights: the (O, l, m) of each key split are
+// written for the solve; attention: out = O sigma / l.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads (A once, then B, C and w
+// tiles through a 3-stage ring), warp 1 owns TMEM and issues the MMAs, warps
+// 2..5 run the exponentials and the epilogue (warp w reads TMEM lanes
+// 32 (w % 4) .. +31, one tile row per thread).  S is double buffered in
+// TMEM (2 x 64 columns), O takes DV columns.  Operands use the 128-byte
+// swizzled canonical layouts: A, B and P K-major, C MN-major.  Every wait is
+// bounded; a wait that runs out records WC_ERR_TIMEOUT and the block winds
+// down (drains its copies and MMAs, frees TMEM) instead of hanging.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include "wc_common.cuh"
+#include "wc_expmm.cuh"
+#include "wc_internal.h"
+#include "wc_tc.cuh"
+
+namespace wc {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128, BN = 64, NS = 3, kThreads = 192;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.0f;  // log2 units: P stays below 2^8 between rescales
+constexpr uint64_t kTcTimeoutNs = 4000000000ull;
+
+struct TcArgs {
+    const int32_t* rank;
+    void* out;
+    const float* wn;     // rownorm: normaliser column, [units][r_pad]
+    const float* sigma;  // rownorm: column scales of the fp16 weights, [units][dv]
+    int* status;
+    int a_rows;          // rows of A per head (r or n_q)
+    int a_head_rows;     // row stride of A between heads in the 2-D view
+    int b_rows;          // rows of B per unit (n or r)
+    int nsplit, split_len;
+    int r, r_pad;
+    int hq, group;
+    float cb;            // beta * log2(e)
+};
+
+template <int D, int DV>
+struct Smem {
+    static constexpr uint32_t A = 0;
+    static constexpr uint32_t kA = BM * D * 2;
+    static constexpr uint32_t kB = BN * D * 2;
+    static constexpr uint32_t kC = BN * DV * 2;
+    static constexpr uint32_t kW = 1024;
+    static constexpr uint32_t kStage = kB + kC + kW;
+    static constexpr uint32_t Stage0 = kA;
+    static constexpr uint32_t P0 = Stage0 + NS * kStage;
+    static constexpr uint32_t kP = BM * BN * 2;
+    static constexpr uint32_t Bar = P0 + 2 * kP;
+    static constexpr uint32_t kTotal = Bar + 256;
+    static constexpr uint32_t kAlloc = kTotal + 1024;  // room to align the base to 1024
+};
+
+template <int D, int DV, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    expmm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                    const __grid_constant__ CUtensorMap mapC, const TcArgs args) {
+    using L = Smem<D, DV>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::Bar);
+    uint64_t* full = bars;            // [NS]
+    uint64_t* empty = bars + NS;      // [NS]
+    uint64_t* a_full = bars + 2 * NS;
+    uint64_t* s_full = a_full + 1;    // [2]
+    uint64_t* s_free = s_full + 2;    // [2]
+    uint64_t* p_full = s_free + 2;    // [2]
+    uint64_t* p_free = p_full + 2;    // [2]
+    uint64_t* drain = p_free + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int z = blockIdx.z;
+    int unit, a_valid, b_lo, b_hi, split = 0, a_row0;
+    if (MODE == kExpmmPartial) {
+        unit = z;
+        a_valid = args.rank[unit];
+        split = blockIdx.y;
+        b_lo = split * args.split_len;
+        b_hi = min(args.b_rows, b_lo + args.split_len);
+        a_row0 = unit * args.a_head_rows + blockIdx.x * BM;
+    } else {
+        const int hkv = args.hq / args.group;
+        unit = (z / args.hq) * hkv + (z % args.hq) / args.group;
+        a_valid = args.a_rows;
+        b_lo = 0;
+        b_hi = args.rank[unit];
+        a_row0 = z * args.a_head_rows + blockIdx.x * BM;
+    }
+    const int a0 = blockIdx.x * BM;
+    if (a0 >= a_valid) return;
+    const int T = b_hi > b_lo ? (b_hi - b_lo + BN - 1) / BN : 0;
+    const int b_row0 = unit * args.b_rows + b_lo;
+
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(a_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&p_free[i], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc<256>(tmem_slot);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && T > 0) {
+            tma_prefetch(&mapA);
+            tma_prefetch(&mapB);
+            tma_prefetch(&mapC);
+            mbar_expect_tx(a_full, L::kA);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tma_load_2d(sm + L::A + c * (BM * 128), &mapA, a_full, c * 64, a_row0);
+            int issued = 0;
+            for (int t = 0; t < T; ++t) {
+                const int s = t % NS;
+                if (t >= NS && !mbar_wait(&empty[s], ((t / NS) - 1) & 1, abort_flag, args.status, kTcTimeoutNs))
+                    break;
+                unsigned char* st = sm + L::Stage0 + s * L::kStage;
+                const uint32_t bytes = L::kB + L::kC + (MODE == kExpmmRownorm ? BN * 4 : 0);
+                mbar_expect_tx(&full[s], bytes);
+                const int brow = b_row0 + t * BN;
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &full[s], c * 64, brow);
+#pragma unroll
+                for (int c = 0; c < DV / 64; ++c)
+                    tma_load_2d(st + L::kB + c * (BN * 128), &mapC, &full[s], c * 64, brow);
+                if (MODE == kExpmmRownorm)
+                    bulk_load(st + L::kB + L::kC, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN, BN * 4,
+                              &full[s]);
+                issued = t + 1;
+            }
+            // wind down: every copy this thread started has landed before the block exits
+            if (*abort_flag) {
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(a_full, 0) && global_ns() - t0 < 100000000ull) {
+                }
+                for (int t = issued - NS > 0 ? issued - NS : 0; t < issued; ++t) {
+                    const int s = t % NS;
+                    const uint64_t t1 = global_ns();
+                    while (!mbar_try_wait(&full[s], (t / NS) & 1) && global_ns() - t1 < 100000000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && T > 0) {
+            constexpr uint32_t idS = idesc_f16(BM, BN, 1, 1, 0, 0);   // bf16 x bf16, both K-major
+            constexpr uint32_t idO = idesc_f16(BM, DV, 0, 0, 0, 1);   // f16 P (K-major) x f16 C (MN-major)
+            const uint32_t sA = smem_u32(sm + L::A);
+            bool ok = mbar_wait(a_full, 0, abort_flag, args.status, kTcTimeoutNs);
+            for (int t = 0; ok && t <= T; ++t) {
+                if (t < T) {
+                    const int s = t % NS, x = t & 1;
+                    ok = mbar_wait(&full[s], (t / NS) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (ok && t >= 2) ok = mbar_wait(&s_free[x], ((t >> 1) - 1) & 1, abort_flag, args.status,
+                                                     kTcTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sB = smem_u32(sm + L::Stage0 + s * L::kStage);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t off = (k & 3) * 32;  // 16 elements = 32 bytes into the 128-byte row
+                        const uint64_t da = sdesc_sw128(sA + (k >> 2) * (BM * 128) + off, 16, 1024);
+                        const uint64_t db = sdesc_sw128(sB + (k >> 2) * (BN * 128) + off, 16, 1024);
+                        mma_f16_ss(tmem + x * BN, da, db, idS, k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[x]);
+                }
+                if (t >= 1) {
+                    const int tp = t - 1, sp = tp % NS, xp = tp & 1;
+                    ok = mbar_wait(&p_full[xp], (tp >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t sP = smem_u32(sm + L::P0 + xp * L::kP);
+                    const uint32_t sC = smem_u32(sm + L::Stage0 + sp * L::kStage + L::kB);
+#pragma unroll
+                    for (int k = 0; k < BN / 16; ++k) {
+                        const uint64_t da = sdesc_sw128(sP + k * 32, 16, 1024);
+                        const uint64_t db = sdesc_sw128(sC + k * (16 * 128), BN * 128, 1024);
+                        mma_f16_ss(tmem + 2 * BN, da, db, idO, (tp > 0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&p_free[xp]);
+                    mma_commit(&empty[sp]);
+                }
+            }
+            // wind down: all issued MMAs complete before TMEM is released
+            mma_commit(drain);
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(drain, 0) && global_ns() - t0 < 1000000000ull) {
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        float m2 = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int t = 0; t < T; ++t) {
+            const int x = t & 1;
+            ok = mbar_wait(&s_full[x], (t >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+            if (!ok) break;
+            tc_fence_after();
+            float s[BN];
+            tmem_ld32(tl + x * BN, s);
+            tmem_ld32(tl + x * BN + 32, s + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[x]);
+
+            const int valid = min(BN, b_hi - (b_lo + t * BN));
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < BN; ++j) {
+                s[j] = j < valid ? s[j] * args.cb : -INFINITY;
+                mt = fmaxf(mt, s[j]);
+            }
+            if (__any_sync(0xffffffffu, mt > m2 + kRescale)) {
+                const float mn = fmaxf(m2, mt);
+                if (t > 0) {
+                    // O holds tiles 0..t-1: wait for the last of them, then rescale in place
+                    ok = mbar_wait(&p_free[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float sc = (m2 == -INFINITY) ? 0.f : ex2(m2 - mn);
+#pragma unroll
+                    for (int c0 = 0; c0 < DV; c0 += 32) {
+                        float o[32];
+                        tmem_ld32(tl + 2 * BN + c0, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= sc;
+                        tmem_st32(tl + 2 * BN + c0, o);
+                    }
+                    tmem_wait_st();
+                    l *= sc;
+                }
+                m2 = mn;
+            }
+            if (t >= 2) {
+                ok = mbar_wait(&p_free[x], ((t - 2) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            const float* wv = reinterpret_cast<const float*>(sm + L::Stage0 + (t % NS) * L::kStage + L::kB + L::kC);
+            unsigned char* prow = sm + L::P0 + x * L::kP + row * 128;
+#pragma unroll
+            for (int c16 = 0; c16 < BN / 8; ++c16) {
+                uint32_t packed[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int j = c16 * 8 + 2 * h;
+                    const float p0 = ex2(s[j] - m2), p1 = ex2(s[j + 1] - m2);
+                    if (MODE == kExpmmRownorm)
+                        l += p0 * wv[j] + p1 * wv[j + 1];
+                    else
+                        l += p0 + p1;
+                    const __half2 hp = __floats2half2_rn(p0, p1);
+                    packed[h] = *reinterpret_cast<const uint32_t*>(&hp);
+                }
+                *reinterpret_cast<uint4*>(prow + ((c16 ^ (row & 7)) << 4)) =
+                    make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[x]);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        float o[DV];
+#pragma unroll
+        for (int c = 0; c < DV; ++c) o[c] = 0.f;
+        if (ok && T > 0) {
+            ok = mbar_wait(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int c0 = 0; c0 < DV; c0 += 32) tmem_ld32(tl + 2 * BN + c0, o + c0);
+                tmem_wait_ld();
+            }
+        }
+        const int a = a0 + row;
+        if (ok && a < a_valid) {
+            if (MODE == kExpmmPartial) {
+                float* dst = static_cast<float*>(args.out) +
+                             (((size_t)unit * args.nsplit + split) * args.r + a) * (DV + 2);
+                // rows are DV + 2 floats apart: 8-byte aligned, not 16
+#pragma unroll
+                for (int c = 0; c < DV; c += 2) *reinterpret_cast<float2*>(dst + c) = make_float2(o[c], o[c + 1]);
+                *reinterpret_cast<float2*>(dst + DV) = make_float2(l, m2 * kLn2);
+            } else {
+                float* dst = static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a) * DV;
+                const float* sg = args.sigma + (size_t)unit * DV;
+                const float inv = 1.f / l;
+#pragma unroll
+                for (int c = 0; c < DV; c += 4)
+                    *reinterpret_cast<float4*>(dst + c) =
+                        make_float4(o[c] * sg[c] * inv, o[c + 1] * sg[c + 1] * inv, o[c + 2] * sg[c + 2] * inv,
+                                    o[c + 3] * sg[c + 3] * inv);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc<256>(tmem);
+}
+
+// V (bf16) -> fp16 copy for the value operand of the weights GEMM.
+__global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, size_t count) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __float2half_rn(__bfloat162float(src[i]));
+}
+
+// Weights for the attention GEMM: per unit and column c < dv, sigma_c =
+// max_s |W[s, c]| and W16[s, c] = W[s, c] / sigma_c (fp16); wn[s] = W[s, dv]
+// padded with zeros to r_pad rows.  One block per unit.
+__global__ void weights_prep_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, __half* W16,
+                                    float* sigma, float* wn, int r, int r_pad, int dv) {
+    const int u = blockIdx.x;
+    const int k = rank[u];
+    const float* Wu = W + (size_t)u * r * (dv + 1);
+    __shared__ float sg[256];
+    for (int c = threadIdx.x; c < dv; c += blockDim.x) {
+        float mx = 0.f;
+        for (int s = 0; s < k; ++s) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
+        sg[c] = mx > 0.f ? mx : 1.f;
+        sigma[(size_t)u * dv + c] = sg[c];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < r * dv; e += blockDim.x) {
+        const int s = e / dv, c = e % dv;
+        const float v = s < k ? Wu[(size_t)s * (dv + 1) + c] / sg[c] : 0.f;
+        W16[(size_t)u * r * dv + e] = __float2half_rn(v);
+    }
+    for (int s = threadIdx.x; s < r_pad; s += blockDim.x) wn[(size_t)u * r_pad + s] = s < k ? Wu[(size_t)s * (dv + 1) + dv] : 0.f;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D row-major view [rows][cols] of 2-byte elements, box = 64 columns x box_rows.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+              uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int DV, int MODE>
+wc_status launch_tc_t(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& C, const TcArgs& a,
+                      dim3 grid, cudaStream_t st) {
+    using L = Smem<D, DV>;
+    auto kern = expmm_tc_kernel<D, DV, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc) != cudaSuccess)
+        return WC_ERR_CUDA;
+    kern<<<grid, kThreads, L::kAlloc, st>>>(A, B, C, a);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+template <int MODE>
+wc_status launch_tc(int d, int dv, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& C,
+                    const TcArgs& a, dim3 grid, cudaStream_t st) {
+    if (d == 64 && dv == 64) return launch_tc_t<64, 64, MODE>(A, B, C, a, grid, st);
+    if (d == 64 && dv == 128) return launch_tc_t<64, 128, MODE>(A, B, C, a, grid, st);
+    if (d == 128 && dv == 64) return launch_tc_t<128, 64, MODE>(A, B, C, a, grid, st);
+    if (d == 128 && dv == 128) return launch_tc_t<128, 128, MODE>(A, B, C, a, grid, st);
+    return WC_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+bool tc_supported(const Shape& s) {
+    return s.dtype == WC_BF16 && (s.d == 64 || s.d == 128) && (s.dv == 64 || s.dv == 128) && encode_fn() != nullptr;
+}
+
+wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K, const void* V,
+                                   const int32_t* rank, char* ws, cudaStream_t st) {
+    const WsLayout Lw = make_layout(s);
+    __half* V16 = reinterpret_cast<__half*>(ws + Lw.v16);
+    const size_t nv = (size_t)s.units * s.n * s.dv;
+    to_half_kernel<<<1184, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(V), V16, nv);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    CUtensorMap mA, mB, mC;
+    if (!make_map(&mA, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BM) ||
+        !make_map(&mB, K, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.n, BN) ||
+        !make_map(&mC, V16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s.dv, (uint64_t)s.units * s.n, BN))
+        return WC_ERR_CUDA;
+    TcArgs a{};
+    a.rank = rank;
+    a.out = ws + Lw.c1part;
+    a.status = reinterpret_cast<int*>(ws + Lw.status);
+    a.a_rows = s.r;
+    a.a_head_rows = s.r;
+    a.b_rows = s.n;
+    a.nsplit = s.nsplit;
+    a.split_len = kSplitKeys;
+    a.r = s.r;
+    a.r_pad = s.r_pad;
+    a.hq = s.hkv;
+    a.group = 1;
+    a.cb = (float)(s.beta * 1.4426950408889634);
+    dim3 grid((s.r + BM - 1) / BM, s.nsplit, s.units);
+    return launch_tc<kExpmmPartial>(s.d, s.dv, mA, mB, mC, a, grid, st);
+}
+
+wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
+                           float* out, char* ws, cudaStream_t st) {
+    const WsLayout Lw = make_layout(s);
+    __half* W16 = reinterpret_cast<__half*>(ws + Lw.w16);
+    float* sigma = reinterpret_cast<float*>(ws + Lw.sigma);
+    float* wn = reinterpret_cast<float*>(ws + Lw.wn);
+    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    CUtensorMap mA, mB, mC;
+    if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
+        !make_map(&mB, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BN) ||
+        !make_map(&mC, W16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s.dv, (uint64_t)s.units * s.r, BN))
+        return WC_ERR_CUDA;
+    TcArgs a{};
+    a.rank = rank;
+    a.out = out;
+    a.wn = wn;
+    a.sigma = sigma;
+    a.status = reinterpret_cast<int*>(ws + Lw.status);
+    a.a_rows = s.nq;
+    a.a_head_rows = s.nq;
+    a.b_rows = s.r;
+    a.nsplit = 1;
+    a.split_len = s.r;
+    a.r = s.r;
+    a.r_pad = s.r_pad;
+    a.hq = s.hq;
+    a.group = s.hq / s.hkv;
+    a.cb = (float)(s.beta * 1.4426950408889634);
+    dim3 grid((s.nq + BM - 1) / BM, 1, s.batch * s.hq);
+    return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
+}
+
+}  // namespace wc

@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
     if ((tid & 31) == 0 && lmax > 0.0) atomicMax(&us->hmax_bits, (unsigned long long)__double_as_longlong(lmax));
+    __syncthreads();  // the scan chunks below span rows that other threads initialised
 
     {
         int lo, hi;
@@ -438,29 +439,40 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     m_max = m_max > (1 << 20) ? (1 << 20) : m_max;
 
     auto kern = rpcholesky_kernel<T>;
-    // occupancy at the largest slice we might use
-    const int c_min = (s.n + m_max - 1) / m_max;
-    int C = c_min;
-    int m = ((s.n + C - 1) / C + kGroup - 1) / kGroup * kGroup;
-    size_t smem = select_smem_bytes(m, s.r, s.d);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem - 1024) != cudaSuccess)
         return WC_ERR_CUDA;
-    int bps = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, kThreads, smem) != cudaSuccess || bps < 1)
-        return WC_ERR_CUDA;
-    const long cap = (long)nsm * bps;
+    auto blocks_per_sm = [&](int m) {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, select_smem_bytes(m, s.r, s.d)) !=
+            cudaSuccess)
+            return 0;
+        return b;
+    };
+    auto rows_for = [&](int C) { return ((s.n + C - 1) / C + kGroup - 1) / kGroup * kGroup; };
 
-    if ((long)s.units * C <= cap) {
-        // spread each unit over more blocks, keeping >= 256 rows per block
-        long want = cap / s.units;
-        const long rows_cap = (s.n + 255) / 256;
-        if (want > rows_cap) want = rows_cap;
-        if (want > kMaxBlocksPerUnit) want = kMaxBlocksPerUnit;
-        if (want > C) C = (int)want;
-        m = ((s.n + C - 1) / C + kGroup - 1) / kGroup * kGroup;
-        C = (s.n + m - 1) / m;
-        smem = select_smem_bytes(m, s.r, s.d);
+    // Most blocks per unit such that every block of the launch is co-resident
+    // (they wait on each other), at >= 256 rows per block; else the fewest
+    // blocks the shared memory allows, in co-resident waves.
+    const int c_min = (s.n + m_max - 1) / m_max;
+    int c_hi = (s.n + 255) / 256;
+    if (c_hi > kMaxBlocksPerUnit) c_hi = kMaxBlocksPerUnit;
+    if (c_hi < c_min) c_hi = c_min;
+    int C = c_min, m = rows_for(c_min);
+    long cap = (long)nsm * blocks_per_sm(m);
+    for (int c = c_hi; c > c_min; --c) {
+        const int mc = rows_for(c);
+        const int ce = (s.n + mc - 1) / mc;
+        const long capc = (long)nsm * blocks_per_sm(mc);
+        if ((long)s.units * ce <= capc) {
+            C = ce;
+            m = mc;
+            cap = capc;
+            break;
+        }
     }
+    C = (s.n + m - 1) / m;
+    const size_t smem = select_smem_bytes(m, s.r, s.d);
+    if (cap < 1) return WC_ERR_CUDA;
     if (C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
 
     SelectArgs a;

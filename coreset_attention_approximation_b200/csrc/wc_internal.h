@@ -34,6 +34,10 @@ struct WsLayout {
     size_t lg;        // float[units][r][r]     gathered L = F[piv, :]
     size_t c1part;    // float[units][nsplit][r][dv + 2]  (O | l | m)
     size_t y;         // double[units][r][dv + 1]
+    size_t v16;       // half[units][n][dv]     values for the tensor-core weights GEMM
+    size_t w16;       // half[units][r][dv]     column-scaled weights for attention
+    size_t sigma;     // float[units][dv]       their column scales
+    size_t wn;        // float[units][r_pad]    normaliser column W[:, dv]
     size_t scratch_end;
     // room for outputs that wc_forward keeps in the workspace when not given
     size_t piv, rank, f, ks, w;
@@ -50,6 +54,7 @@ struct Shape {
     int32_t units;         // batch * hkv
     int32_t esize;         // bytes per Q/K/V element
     int32_t nsplit;        // C1 partial sums
+    int32_t r_pad;         // r rounded up to 64
 };
 
 wc_status make_shape(const wc_shape* in, Shape* out);
@@ -66,5 +71,12 @@ wc_status launch_solve(const Shape& s, const int32_t* rank, float* W, char* ws, 
 wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const float* W,
                         const int32_t* rank, float* out, char* ws, cudaStream_t st);
 wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st);
+
+// Tensor-core path (bf16 inputs, d and dv in {64, 128}).
+bool tc_supported(const Shape& s);
+wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K, const void* V,
+                                   const int32_t* rank, char* ws, cudaStream_t st);
+wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
+                           float* out, char* ws, cudaStream_t st);
 
 }  // namespace wc

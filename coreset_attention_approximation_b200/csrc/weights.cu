@@ -198,6 +198,7 @@ wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const
 
 wc_status launch_coreset_values(const Shape& s, const void* Ks, const void* K, const void* V, const int32_t* rank,
                                 char* ws, cudaStream_t st) {
+    if (tc_supported(s)) return launch_coreset_values_tc(s, Ks, K, V, rank, ws, st);
     const WsLayout L = make_layout(s);
     ExpmmArgs e{};
     e.A = Ks; e.a_stride = (int64_t)s.r * s.d; e.a_rows = s.r;

@@ -154,3 +154,29 @@ def test_full_long_workload_prefix_and_properties():
     k = int(rank[0, 0])
     out_o = oracle.coreset_attend(Q[0, 0, qs], res["Ks"][0, 0, :k], res["W"][0, 0, :k], beta)
     assert rel_err(res["out"][0, 0, qs].numpy(), out_o) <= TOL_OUT[torch.bfloat16]
+
+
+def test_running_max_rescale_large_dynamic_range():
+    """One key with a much larger norm than the rest is drawn first; in the
+    weights GEMM its row meets its own (largest) logit only in a late key
+    tile, so the running maximum grows by far more than the rescale
+    threshold mid-row."""
+    g = torch.Generator().manual_seed(7)
+    n, d, dv, nq = 520, 64, 64, 200
+    K = torch.randn(1, 1, n, d, generator=g) * 0.3
+    # |k_500|^2 / sqrt(d) = 8 (11.5 in log2 units) against cross logits of about 1
+    K[0, 0, 500] = 8.0 * torch.nn.functional.normalize(torch.randn(d, generator=g), dim=0)
+    V = torch.randn(1, 1, n, dv, generator=g)
+    Q = torch.randn(1, 1, nq, d, generator=g) * 0.3
+    Q[0, 0, :20] = 0.5 * K[0, 0, 500]
+    Q, K, V = Q.to(torch.bfloat16), K.to(torch.bfloat16), V.to(torch.bfloat16)
+    compare(Q, K, V, 48, seed=1)
+    res = run_gpu(Q, K, V, 48, seed=1)
+    assert int(res["piv"][0, 0, 0]) == 500 and int(res["rank"][0, 0]) == 48
+
+
+@pytest.mark.parametrize("d,dv", [(32, 96), (128, 64), (64, 128)])
+def test_other_head_widths_bf16(d, dv):
+    # (32, 96) runs on CUDA cores, the others on the tensor-core kernel
+    w = WORKLOADS["vit"].replace(batch=1, hq=4, hkv=2, n_k=1500, n_q=300, d=d, dv=dv, r=100)
+    compare(*make_inputs(w, seed=d + dv), w.r, seed=3)
