@@ -491,4 +491,36 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
 }
 
+// Attention on the tensor cores with caller-chosen scratch pointers (status
+// word, fp16 weights, column scales, normaliser column); used by the entry
+// point that allocates nothing.
+wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
+                              float* out, int* status, __half* W16, float* sigma, float* wn, cudaStream_t st) {
+    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    CUtensorMap mA, mB, mC;
+    if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
+        !make_map(&mB, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BN) ||
+        !make_map(&mC, W16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s.dv, (uint64_t)s.units * s.r, BN))
+        return WC_ERR_CUDA;
+    TcArgs a{};
+    a.rank = rank;
+    a.out = out;
+    a.wn = wn;
+    a.sigma = sigma;
+    a.status = status;
+    a.a_rows = s.nq;
+    a.a_head_rows = s.nq;
+    a.b_rows = s.r;
+    a.nsplit = 1;
+    a.split_len = s.r;
+    a.r = s.r;
+    a.r_pad = s.r_pad;
+    a.hq = s.hq;
+    a.group = s.hq / s.hkv;
+    a.cb = (float)(s.beta * 1.4426950408889634);
+    dim3 grid((s.nq + BM - 1) / BM, 1, s.batch * s.hq);
+    return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
+}
+
 }  // namespace wc

@@ -1,6 +1,7 @@
 // wc_internal.h — workspace layout and kernel launchers of the WildCat library.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -78,5 +79,7 @@ wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K
                                    const int32_t* rank, char* ws, cudaStream_t st);
 wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
                            float* out, char* ws, cudaStream_t st);
+wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
+                              float* out, int* status, __half* W16, float* sigma, float* wn, cudaStream_t st);
 
 }  // namespace wc

@@ -42,6 +42,7 @@ class WcShape(ctypes.Structure):
 EXPORTS = [
     "wc_f_ld", "wc_workspace_bytes", "wc_forward_workspace_bytes", "wc_select", "wc_weights", "wc_attend",
     "wc_forward", "wc_check_device_status", "wc_selftest_wait_timeout", "wc_status_string",
+    "wc_attend_noalloc",
 ]
 
 _lib = None
@@ -69,6 +70,7 @@ def lib():
         L.wc_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
         L.wc_selftest_wait_timeout.restype = i32
         L.wc_status_string.argtypes, L.wc_status_string.restype = [i32], ctypes.c_char_p
+        L.wc_attend_noalloc.argtypes, L.wc_attend_noalloc.restype = [sp, vp, vp, vp, vp, vp, vp], i32
         _lib = L
     return _lib
 
@@ -160,6 +162,19 @@ def attend(Q, Ks, W, rank, n_k, *, ws=None, stream=None, **kw):
     ws = workspace(shape, Q.device) if ws is None else ws
     _check(lib().wc_attend(ctypes.byref(shape), _ptr(Q), _ptr(Ks), _ptr(W), _ptr(rank), _ptr(out),
                            _ptr(ws), ws.numel(), _stream(stream)), "wc_attend")
+    return out
+
+
+def attend_noalloc(Q, Ks, W, rank, n_k, *, out=None, stream=None, **kw):
+    """wc_attend_noalloc: attention with the library's fixed device scratch,
+    for callers that cannot allocate.  `out` may be preallocated."""
+    B, Hq, nq, d = Q.shape
+    Hkv, r, dv = Ks.shape[1], Ks.shape[2], W.shape[-1] - 1
+    shape = make_shape(B, Hq, Hkv, n_k, nq, d, dv, r, Q.dtype, **kw)
+    if out is None:
+        out = torch.empty(B, Hq, nq, dv, dtype=torch.float32, device=Q.device)
+    _check(lib().wc_attend_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(Ks), _ptr(W), _ptr(rank), _ptr(out),
+                                   _stream(stream)), "wc_attend_noalloc")
     return out
 
 

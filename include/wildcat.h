@@ -149,6 +149,31 @@ wc_status wc_check_device_status(void* ws, void* stream);
  */
 wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_ms, void* stream);
 
+/*
+ * attend_noalloc — the same result as wc_attend, for callers that cannot
+ * allocate device memory or pass a workspace (an allocator that must not be
+ * re-entered, a process whose memory budget is fixed up front, a plugin that
+ * only receives its tensors).  The paper has no counterpart; this is a
+ * deployment variant of the attend step.
+ *   - Scratch: a fixed 16 MiB array in device memory owned by the library
+ *     (every GPU that loads the library holds it until the process exits).
+ *     Shapes that need more (2 * units * r * dv + 4 * units * (dv + r rounded
+ *     up to 64) bytes, plus alignment) are refused with WC_ERR_WORKSPACE
+ *     before any launch.  bf16 inputs with d, dv in {64, 128} use it; other
+ *     shapes run on the CUDA-core kernel, which needs no scratch.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ *   - Every call shares the one array and leaves its contents behind; the
+ *     call clears what it needs cleared.  Calls whose execution overlaps on
+ *     the GPU (other streams, other threads) race on it: serialise them.
+ *   - A device-side wait that runs out ends the kernel cleanly but is not
+ *     reported here (use wc_attend with a workspace to read such errors).
+ */
+wc_status wc_attend_noalloc(const wc_shape* shape, const void* Q, const void* Ks, const float* W,
+                            const int32_t* rank, float* out, void* stream);
+
 /* Static text for a status code. */
 const char* wc_status_string(wc_status status);
 
