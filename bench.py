@@ -305,6 +305,8 @@ def run_ours(args, world, rank, local):
     if wildcat.check_device_status(ws) != 0:
         raise RuntimeError("device status after e2e steps")
 
+    kernels = kernel_breakdown(step)
+
     peaks, which = load_peaks()
     sel_avg = sum(sel_ms) / len(sel_ms)
     sb = select_bytes(w)
@@ -339,13 +341,8 @@ def run_ours(args, world, rank, local):
             "algorithmic_bytes_per_launch": sb, "launch_ms": sel_avg,
         },
         "stages_ms": {"select": sel_avg, "weights": wts_avg, "attend": att_avg},
-        "gemm": {
-            "weights_tflops": f1 / (wts_avg * 1e-3) / 1e12, "attend_tflops": f2 / (att_avg * 1e-3) / 1e12,
-            "peak_tflops_bf16": peaks["bf16_tflops"],
-            "weights_frac": f1 / (wts_avg * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            "attend_frac": f2 / (att_avg * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            "note": "weights stage includes the gather and the fp64 solve",
-        },
+        "gemm": gemm_report(kernels, f1, f2, peaks),
+        "kernels_ms": kernels,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
@@ -354,8 +351,50 @@ def run_ours(args, world, rank, local):
     return res
 
 
-# select (1 cooperative wave here), gather, C1 exp-GEMM, solve, attend exp-GEMM
-LAUNCHES_PER_STEP = 5
+# select (1 cooperative wave here), gather, fp16 copy of V, C1 exp-GEMM, merge of
+# the C1 partials, triangular solves, weight preparation, attention exp-GEMM
+LAUNCHES_PER_STEP = 8
+
+
+def kernel_breakdown(step):
+    """Device time of each kernel of one extra step (outside the timed
+    region), from CUPTI activity records via torch.profiler."""
+    from torch.profiler import ProfilerActivity, profile
+
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize()
+    import re
+
+    out = {}
+    for ev in prof.events():
+        if ev.device_type.name != "CUDA":
+            continue
+        name = ev.name
+        short = None
+        m = re.search(r"expmm_(tc|simt)_kernel<[^>]*?(\d)>", name)
+        if m:
+            short = ("weights_gemm", "attend_gemm")[int(m.group(2))]
+        else:
+            for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
+                             ("merge_c1", "merge_c1"), ("trsv_kernel", "solve"), ("weights_prep", "w_prep")):
+                if key in name:
+                    short = tag
+                    break
+        if short:
+            out[short] = out.get(short, 0.0) + ev.device_time / 1e3
+    return out
+
+
+def gemm_report(kernels, f1, f2, peaks):
+    rep = {"peak_tflops_bf16": peaks["bf16_tflops"], "peak_tflops_bf16_sustained": peaks.get("bf16_tflops_sustained")}
+    for name, flops in (("weights_gemm", f1), ("attend_gemm", f2)):
+        ms = kernels.get(name)
+        if ms:
+            tf = flops / (ms * 1e-3) / 1e12
+            rep[name] = {"ms": ms, "tflops": tf, "frac": tf / peaks["bf16_tflops"], "flops": flops}
+    return rep
 
 
 def run_reference(args, world, rank):

@@ -34,7 +34,7 @@ struct WsLayout {
     size_t kt;        // dtype[units][d][ldf]   transposed keys
     size_t lg;        // float[units][r][r]     gathered L = F[piv, :]
     size_t c1part;    // float[units][nsplit][r][dv + 2]  (O | l | m)
-    size_t y;         // double[units][r][dv + 1]
+    size_t y;         // double[units][dv + 1][r]  C1, column-major, solved in place
     size_t v16;       // half[units][n][dv]     values for the tensor-core weights GEMM
     size_t w16;       // half[units][r][dv]     column-scaled weights for attention
     size_t sigma;     // float[units][dv]       their column scales

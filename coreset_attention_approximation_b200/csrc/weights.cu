@@ -5,7 +5,7 @@
 // compressed as V_S = W V.  Here the weights act on [V | 1], so the softmax
 // normaliser is compressed with the values:
 //   C1 = exp(beta K_S K^T) [V | 1]           (gather + exp-GEMM, split over keys)
-//   W  = L^-T (L^-1 C1),  L = F[piv, :rank]  (blocked fp64 triangular solves)
+//   W  = L^-T (L^-1 C1),  L = F[piv, :rank]  (fp64 triangular solves, a warp per 4 columns)
 // L L^T = h(K_S, K_S) because the pivot rows of the RPCholesky factor are the
 // Cholesky factor of the kernel matrix on the coreset (in pivot order).
 #include "wc_common.cuh"
@@ -33,150 +33,140 @@ __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict
         lrow[b] = (p >= 0 && b <= a) ? Fu[(int64_t)b * ldf + p] : 0.f;
 }
 
-constexpr int kTile = 32;      // rows per solve block / columns per solve CTA
-constexpr int kSolveThreads = 256;
+constexpr int kCols = 4;  // right-hand-side columns per solving warp
 
-// Merge the C1 partials of row a, column c (fp64): sum_s e^{m_s} O_s.
-__device__ __forceinline__ double merged_c1(const float* part, int nsplit, int r, int dv, int a, int c) {
-    const int w = dv + 2;
+// C1 from the partial sums of the key splits, in fp64:
+//   C1[a, c] = e^M sum_s e^{m_s - M} O_s[a, c],  M = max_s m_s
+// written column-major, Ct[u, c, a], for the solves.  One block per (a, u).
+__global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t* __restrict__ rank, double* Ct,
+                                int nsplit, int r, int dv) {
+    const int a = blockIdx.x, u = blockIdx.y;
+    if (a >= rank[u]) return;
+    const int w = dv + 2, wcols = dv + 1;
+    const float* part = c1part + (size_t)u * nsplit * r * w;
     double mx = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) mx = fmax(mx, (double)part[((size_t)s * r + a) * w + dv + 1]);
-    if (!(mx > -INFINITY)) return 0.0;
-    double acc = 0.0;
-    for (int s = 0; s < nsplit; ++s) {
-        const float* row = part + ((size_t)s * r + a) * w;
-        const double ms = (double)row[dv + 1];
-        if (ms > -INFINITY) acc += exp(ms - mx) * (double)row[c];
+    for (int sp = 0; sp < nsplit; ++sp) mx = fmax(mx, (double)part[((size_t)sp * r + a) * w + dv + 1]);
+    for (int c = threadIdx.x; c < wcols; c += blockDim.x) {
+        double acc = 0.0;
+        if (mx > -INFINITY) {
+            for (int sp = 0; sp < nsplit; ++sp) {
+                const float* row = part + ((size_t)sp * r + a) * w;
+                const double ms = (double)row[dv + 1];
+                if (ms > -INFINITY) acc += exp(ms - mx) * (double)row[c];
+            }
+            acc *= exp(mx);
+        }
+        Ct[((size_t)u * wcols + c) * r + a] = acc;
     }
-    return acc * exp(mx);
 }
 
-// One block per (column tile, unit): forward then backward substitution on
-// kTile columns of C1, in kTile x kTile blocks, fp64 throughout.
-__global__ void __launch_bounds__(kSolveThreads) solve_kernel(const float* __restrict__ c1part,
-                                                              const float* __restrict__ Lg,
-                                                              const int32_t* __restrict__ rank, double* Y,
-                                                              float* W, int nsplit, int r, int dv) {
+// W = L^-T (L^-1 C1) for kCols right-hand sides of one unit, one warp, fp64,
+// in blocks of 32 rows.  Forward, block [a0, a0+32): lane i owns row a0+i,
+// subtracts L[a0+i, :a0] y[:a0] (its own row of L, independent loads), then the
+// 32 x 32 diagonal block is solved through shuffles.  Backward, blocks from the
+// last: lane i owns entry a0+i, subtracts sum_{b >= a0+32} L[b, a0+i] x_b (row
+// segments of L, coalesced across the warp), then the diagonal block.
+// y / x live in shared memory, [kCols][r].
+__global__ void __launch_bounds__(32) trsv_kernel(const float* __restrict__ Lg, const int32_t* __restrict__ rank,
+                                                  const double* __restrict__ Ct, float* W, int r, int dv) {
+    extern __shared__ double ys[];
     const int u = blockIdx.y;
-    const int c0 = blockIdx.x * kTile;
     const int wcols = dv + 1;
-    const int ncol = min(kTile, wcols - c0);
+    const int c0 = blockIdx.x * kCols;
+    const int nc = min(kCols, wcols - c0);
     const int k = rank[u];
     const float* L = Lg + (size_t)u * r * r;
-    const float* part = c1part + (size_t)u * nsplit * r * (dv + 2);
-    double* Yu = Y + (size_t)u * r * wcols;
+    const double* C = Ct + (size_t)u * wcols * r;
     float* Wu = W + (size_t)u * r * wcols;
-    const int tid = threadIdx.x;
+    const int lane = threadIdx.x;
 
-    __shared__ double Ls[kTile][kTile + 1];
-    __shared__ double Ys[kTile][kTile + 1];
-    __shared__ double Yd[kTile][kTile + 1];  // the diagonal block being solved
-
-    // thread -> (row ra, columns ca + 8q)
-    const int ra = tid / 8, ca = tid % 8;
-
-    // ---- forward: L Y = C1
-    for (int a0 = 0; a0 < k; a0 += kTile) {
-        const int rows = min(kTile, k - a0);
-        double acc[4];
+    // ---- forward: L y = c
+    for (int a0 = 0; a0 < k; a0 += 32) {
+        const int a = a0 + lane;
+        const bool live = a < k;
+        double acc[kCols];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int c = ca + 8 * q;
-            acc[q] = (ra < rows && c < ncol) ? merged_c1(part, nsplit, r, dv, a0 + ra, c0 + c) : 0.0;
-        }
-        for (int b0 = 0; b0 < a0; b0 += kTile) {
-            for (int e = tid; e < kTile * kTile; e += kSolveThreads) {
-                const int i = e / kTile, jj = e % kTile;
-                Ls[i][jj] = (i < rows) ? (double)L[(size_t)(a0 + i) * r + b0 + jj] : 0.0;
-                Ys[i][jj] = (jj < ncol) ? Yu[(size_t)(b0 + i) * wcols + c0 + jj] : 0.0;
+        for (int q = 0; q < kCols; ++q) acc[q] = (live && q < nc) ? C[(size_t)(c0 + q) * r + a] : 0.0;
+        float lb[32];  // this row's entries in the diagonal block
+        if (live) {
+            const float* La = L + (size_t)a * r;
+#pragma unroll 8
+            for (int b = 0; b < a0; ++b) {
+                const double l = (double)La[b];
+#pragma unroll
+                for (int q = 0; q < kCols; ++q) acc[q] -= l * ys[q * r + b];
             }
-            __syncthreads();
-#pragma unroll 4
-            for (int b = 0; b < kTile; ++b) {
-                const double l = Ls[ra][b];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc[q] -= l * Ys[b][ca + 8 * q];
-            }
-            __syncthreads();
-        }
-        // diagonal block
-        for (int e = tid; e < kTile * kTile; e += kSolveThreads) {
-            const int i = e / kTile, jj = e % kTile;
-            Ls[i][jj] = (i < rows && jj < rows) ? (double)L[(size_t)(a0 + i) * r + a0 + jj] : 0.0;
-        }
+            for (int t = 0; t < 32; ++t) lb[t] = (a0 + t < k) ? La[a0 + t] : 0.f;
+        } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) Yd[ra][ca + 8 * q] = acc[q];
-        __syncthreads();
-        if (tid < ncol) {
-            for (int i = 0; i < rows; ++i) {
-                double v = Yd[i][tid];
-                for (int b = 0; b < i; ++b) v -= Ls[i][b] * Yd[b][tid];
-                Yd[i][tid] = v / Ls[i][i];
+            for (int t = 0; t < 32; ++t) lb[t] = 0.f;
+        }
+        const int rows = min(32, k - a0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i < rows) {
+                double yi[kCols];
+#pragma unroll
+                for (int q = 0; q < kCols; ++q) {
+                    const double v = (lane == i) ? acc[q] / (double)lb[i] : 0.0;
+                    yi[q] = __shfl_sync(0xffffffffu, v, i);
+                }
+                if (lane == i) {
+#pragma unroll
+                    for (int q = 0; q < kCols; ++q) ys[q * r + a] = yi[q];
+                }
+                if (lane > i) {
+                    const double l = (double)lb[i];
+#pragma unroll
+                    for (int q = 0; q < kCols; ++q) acc[q] -= l * yi[q];
+                }
             }
         }
-        __syncthreads();
-        for (int e = tid; e < rows * ncol; e += kSolveThreads) {
-            const int i = e / ncol, c = e % ncol;
-            Yu[(size_t)(a0 + i) * wcols + c0 + c] = Yd[i][c];
-        }
-        __syncthreads();
+        __syncwarp();
     }
 
-    // ---- backward: L^T W = Y, blocks from the last
-    const int nblk = (k + kTile - 1) / kTile;
-    for (int bi = nblk - 1; bi >= 0; --bi) {
-        const int a0 = bi * kTile;
-        const int rows = min(kTile, k - a0);
-        double acc[4];
+    // ---- backward: L^T x = y
+    for (int a0 = (k - 1) / 32 * 32; k > 0 && a0 >= 0; a0 -= 32) {
+        const int a = a0 + lane;
+        const bool live = a < k;
+        double acc[kCols];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int c = ca + 8 * q;
-            acc[q] = (ra < rows && c < ncol) ? Yu[(size_t)(a0 + ra) * wcols + c0 + c] : 0.0;
-        }
-        for (int b0 = a0 + kTile; b0 < k; b0 += kTile) {
-            const int brows = min(kTile, k - b0);
-            for (int e = tid; e < kTile * kTile; e += kSolveThreads) {
-                const int i = e / kTile, jj = e % kTile;
-                // Ls[i][jj] = L[b0 + jj][a0 + i]  (transposed block)
-                Ls[i][jj] = (i < rows && jj < brows) ? (double)L[(size_t)(b0 + jj) * r + a0 + i] : 0.0;
-                Ys[i][jj] = (i < brows && jj < ncol) ? Yu[(size_t)(b0 + i) * wcols + c0 + jj] : 0.0;
-            }
-            __syncthreads();
-#pragma unroll 4
-            for (int b = 0; b < kTile; ++b) {
-                const double l = Ls[ra][b];
+        for (int q = 0; q < kCols; ++q) acc[q] = live ? ys[q * r + a] : 0.0;
+#pragma unroll 8
+        for (int b = a0 + 32; b < k; ++b) {
+            const double l = live ? (double)L[(size_t)b * r + a] : 0.0;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc[q] -= l * Ys[b][ca + 8 * q];
-            }
-            __syncthreads();
+            for (int q = 0; q < kCols; ++q) acc[q] -= l * ys[q * r + b];
         }
-        for (int e = tid; e < kTile * kTile; e += kSolveThreads) {
-            const int i = e / kTile, jj = e % kTile;
-            Ls[i][jj] = (i < rows && jj < rows) ? (double)L[(size_t)(a0 + i) * r + a0 + jj] : 0.0;
-        }
+        float lt[32];  // lt[i] = L[a0 + i, a]: this entry's column of the diagonal block
 #pragma unroll
-        for (int q = 0; q < 4; ++q) Yd[ra][ca + 8 * q] = acc[q];
-        __syncthreads();
-        if (tid < ncol) {
-            for (int i = rows - 1; i >= 0; --i) {
-                double v = Yd[i][tid];
-                for (int b = i + 1; b < rows; ++b) v -= Ls[b][i] * Yd[b][tid];
-                Yd[i][tid] = v / Ls[i][i];
+        for (int i = 0; i < 32; ++i) lt[i] = (live && a0 + i < k) ? L[(size_t)(a0 + i) * r + a] : 0.f;
+        const int rows = min(32, k - a0);
+#pragma unroll
+        for (int i = 31; i >= 0; --i) {
+            if (i < rows) {
+                double xi[kCols];
+#pragma unroll
+                for (int q = 0; q < kCols; ++q) {
+                    const double v = (lane == i) ? acc[q] / (double)lt[i] : 0.0;
+                    xi[q] = __shfl_sync(0xffffffffu, v, i);
+                }
+                if (lane == i) {
+#pragma unroll
+                    for (int q = 0; q < kCols; ++q) ys[q * r + a] = xi[q];
+                }
+                if (lane < i) {
+                    const double l = (double)lt[i];
+#pragma unroll
+                    for (int q = 0; q < kCols; ++q) acc[q] -= l * xi[q];
+                }
             }
         }
-        __syncthreads();
-        for (int e = tid; e < rows * ncol; e += kSolveThreads) {
-            const int i = e / ncol, c = e % ncol;
-            Yu[(size_t)(a0 + i) * wcols + c0 + c] = Yd[i][c];
-            Wu[(size_t)(a0 + i) * wcols + c0 + c] = (float)Yd[i][c];
-        }
-        __syncthreads();
+        __syncwarp();
     }
-    // rows >= rank are zero
-    for (int e = tid; e < (r - k) * ncol; e += kSolveThreads) {
-        const int i = k + e / ncol, c = e % ncol;
-        Wu[(size_t)i * wcols + c0 + c] = 0.f;
-    }
+    for (int q = 0; q < nc; ++q)
+        for (int a = lane; a < r; a += 32) Wu[(size_t)a * wcols + c0 + q] = a < k ? (float)ys[q * r + a] : 0.f;
 }
 
 }  // namespace
@@ -217,10 +207,15 @@ wc_status launch_coreset_values(const Shape& s, const void* Ks, const void* K, c
 
 wc_status launch_solve(const Shape& s, const int32_t* rank, float* W, char* ws, cudaStream_t st) {
     const WsLayout L = make_layout(s);
-    dim3 grid((s.dv + 1 + kTile - 1) / kTile, s.units);
-    solve_kernel<<<grid, kSolveThreads, 0, st>>>(reinterpret_cast<const float*>(ws + L.c1part),
-                                                 reinterpret_cast<const float*>(ws + L.lg), rank,
-                                                 reinterpret_cast<double*>(ws + L.y), W, s.nsplit, s.r, s.dv);
+    double* Ct = reinterpret_cast<double*>(ws + L.y);
+    merge_c1_kernel<<<dim3(s.r, s.units), 160, 0, st>>>(reinterpret_cast<const float*>(ws + L.c1part), rank, Ct,
+                                                        s.nsplit, s.r, s.dv);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    const size_t smem = sizeof(double) * kCols * (size_t)s.r;
+    if (cudaFuncSetAttribute(trsv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return WC_ERR_CUDA;
+    trsv_kernel<<<dim3((s.dv + 1 + kCols - 1) / kCols, s.units), 32, smem, st>>>(
+        reinterpret_cast<const float*>(ws + L.lg), rank, Ct, W, s.r, s.dv);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
