@@ -33,7 +33,13 @@ namespace {
 
 using namespace tc;
 
-constexpr int BM = 128, BN = 64, NS = 3, kThreads = 192;
+constexpr int BM = 128;              // rows per CTA (one TMEM lane per row)
+constexpr int TILES = 1;             // row tiles per CTA
+constexpr int BN = 128;              // keys per stage
+constexpr int NB = 3;                // key-tile stages: released once S is computed
+constexpr int NC = 3;                // value-tile stages: released once PV is computed
+// warps: 0 key loader, 1 value loader, 2 S issuer, 3 PV issuer, 4..7 softmax
+constexpr int kThreads = 256;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // log2 units: P stays below 2^8 between rescales
 constexpr uint64_t kTcTimeoutNs = 4000000000ull;
@@ -55,20 +61,20 @@ struct TcArgs {
 
 template <int D, int DV>
 struct Smem {
+    static constexpr uint32_t kA = BM * D * 2;         // the row tile of A
+    static constexpr uint32_t kB = BN * D * 2;         // one key tile (1024-aligned: swizzle atoms)
+    static constexpr uint32_t kC = BN * DV * 2;        // one value tile
     static constexpr uint32_t A = 0;
-    static constexpr uint32_t kA = BM * D * 2;
-    static constexpr uint32_t kB = BN * D * 2;
-    static constexpr uint32_t kC = BN * DV * 2;
-    static constexpr uint32_t kW = 1024;
-    static constexpr uint32_t kStage = kB + kC + kW;
-    static constexpr uint32_t Stage0 = kA;
-    static constexpr uint32_t P0 = Stage0 + NS * kStage;
-    static constexpr uint32_t kP = BM * BN * 2;
-    static constexpr uint32_t Bar = P0 + 2 * kP;
+    static constexpr uint32_t B0 = kA;                  // [NB] key tiles
+    static constexpr uint32_t C0 = B0 + NB * kB;        // [NC] value tiles
+    static constexpr uint32_t Wv = C0 + NC * kC;        // [NC][BN] normaliser weights (rownorm)
+    static constexpr uint32_t Bar = Wv + NC * BN * 4;
     static constexpr uint32_t kTotal = Bar + 256;
-    static constexpr uint32_t kAlloc = kTotal + 1024;  // room to align the base to 1024
+    static constexpr uint32_t kAlloc = kTotal + 1024;   // room to align the base to 1024
 };
 
+// TMEM: S / P buffer x (x = key block & 1) at columns 128 x .. +127 (P as fp16
+// pairs over the first 64 columns of the S it came from), O at 256 .. 256+DV-1.
 template <int D, int DV, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     expmm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
@@ -78,15 +84,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::Bar);
-    uint64_t* full = bars;            // [NS]
-    uint64_t* empty = bars + NS;      // [NS]
-    uint64_t* a_full = bars + 2 * NS;
-    uint64_t* s_full = a_full + 1;    // [2]
-    uint64_t* s_free = s_full + 2;    // [2]
-    uint64_t* p_full = s_free + 2;    // [2]
-    uint64_t* p_free = p_full + 2;    // [2]
-    uint64_t* drain = p_free + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* fullB = bars;                   // [NB]
+    uint64_t* emptyB = fullB + NB;            // [NB]
+    uint64_t* fullC = emptyB + NB;            // [NC]
+    uint64_t* emptyC = fullC + NC;            // [NC]
+    uint64_t* a_full = emptyC + NC;
+    uint64_t* s_full = a_full + 1;            // [2]
+    uint64_t* p_full = s_full + 2;            // [2]
+    uint64_t* p_free = p_full + 2;            // [2]
+    uint64_t* drain = p_free + 2;             // [2] (S issuer, PV issuer)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -113,147 +120,176 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b_row0 = unit * args.b_rows + b_lo;
 
     if (tid == 0) {
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
+        for (int i = 0; i < NB; ++i) {
+            mbar_init(&fullB[i], 1);
+            mbar_init(&emptyB[i], 1);
+        }
+        for (int i = 0; i < NC; ++i) {
+            mbar_init(&fullC[i], 1);
+            mbar_init(&emptyC[i], 1);
         }
         mbar_init(a_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
-            mbar_init(&p_full[i], 4);
-            mbar_init(&p_free[i], 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 4);
+            mbar_init(&p_free[x], 1);
+            mbar_init(&drain[x], 1);
         }
-        mbar_init(drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 1) tmem_alloc<256>(tmem_slot);
+    if (warp == 2) tmem_alloc<512>(tmem_slot);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint32_t tO0 = tmem + 2 * BN;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+    if (warp <= 1) {
+        // ------------------------------------------------------------ TMA producers
+        // warp 0 loads A once, then the key tiles; warp 1 the value tiles (and w)
+        const bool keys = warp == 0;
         if (lane == 0 && T > 0) {
-            tma_prefetch(&mapA);
-            tma_prefetch(&mapB);
-            tma_prefetch(&mapC);
-            mbar_expect_tx(a_full, L::kA);
+            if (keys) {
+                tma_prefetch(&mapA);
+                tma_prefetch(&mapB);
+                mbar_expect_tx(a_full, L::kA);
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) tma_load_2d(sm + L::A + c * (BM * 128), &mapA, a_full, c * 64, a_row0);
+                for (int c = 0; c < D / 64; ++c) tma_load_2d(sm + L::A + c * (BM * 128), &mapA, a_full, c * 64, a_row0);
+            } else {
+                tma_prefetch(&mapC);
+            }
+            const int NR = keys ? NB : NC;
+            uint64_t* fl = keys ? fullB : fullC;
+            uint64_t* em = keys ? emptyB : emptyC;
             int issued = 0;
             for (int t = 0; t < T; ++t) {
-                const int s = t % NS;
-                if (t >= NS && !mbar_wait(&empty[s], ((t / NS) - 1) & 1, abort_flag, args.status, kTcTimeoutNs))
+                const int s = t % NR;
+                if (t >= NR && !mbar_wait(&em[s], ((t / NR) - 1) & 1, abort_flag, args.status, kTcTimeoutNs))
                     break;
-                unsigned char* st = sm + L::Stage0 + s * L::kStage;
-                const uint32_t bytes = L::kB + L::kC + (MODE == kExpmmRownorm ? BN * 4 : 0);
-                mbar_expect_tx(&full[s], bytes);
                 const int brow = b_row0 + t * BN;
+                if (keys) {
+                    mbar_expect_tx(&fl[s], L::kB);
+                    unsigned char* st = sm + L::B0 + s * L::kB;
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &full[s], c * 64, brow);
+                    for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &fl[s], c * 64, brow);
+                } else {
+                    mbar_expect_tx(&fl[s], L::kC + (MODE == kExpmmRownorm ? BN * 4 : 0));
+                    unsigned char* st = sm + L::C0 + s * L::kC;
 #pragma unroll
-                for (int c = 0; c < DV / 64; ++c)
-                    tma_load_2d(st + L::kB + c * (BN * 128), &mapC, &full[s], c * 64, brow);
-                if (MODE == kExpmmRownorm)
-                    bulk_load(st + L::kB + L::kC, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN, BN * 4,
-                              &full[s]);
+                    for (int c = 0; c < DV / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapC, &fl[s], c * 64, brow);
+                    if (MODE == kExpmmRownorm)
+                        bulk_load(sm + L::Wv + s * BN * 4, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN,
+                                  BN * 4, &fl[s]);
+                }
                 issued = t + 1;
             }
             // wind down: every copy this thread started has landed before the block exits
             if (*abort_flag) {
                 const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(a_full, 0) && global_ns() - t0 < 100000000ull) {
+                while (keys && !mbar_try_wait(a_full, 0) && global_ns() - t0 < 100000000ull) {
                 }
-                for (int t = issued - NS > 0 ? issued - NS : 0; t < issued; ++t) {
-                    const int s = t % NS;
+                for (int t = issued - NR > 0 ? issued - NR : 0; t < issued; ++t) {
                     const uint64_t t1 = global_ns();
-                    while (!mbar_try_wait(&full[s], (t / NS) & 1) && global_ns() - t1 < 100000000ull) {
+                    while (!mbar_try_wait(&fl[t % NR], (t / NR) & 1) && global_ns() - t1 < 100000000ull) {
                     }
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ S issuer: S(t) = A B_t^T into buffer t & 1
         if (lane == 0 && T > 0) {
             constexpr uint32_t idS = idesc_f16(BM, BN, 1, 1, 0, 0);   // bf16 x bf16, both K-major
-            constexpr uint32_t idO = idesc_f16(BM, DV, 0, 0, 0, 1);   // f16 P (K-major) x f16 C (MN-major)
-            const uint32_t sA = smem_u32(sm + L::A);
+            const uint64_t dA = sdesc_sw128(smem_u32(sm + L::A), 16, 1024);
+            const uint64_t dB = sdesc_sw128(smem_u32(sm + L::B0), 16, 1024);
             bool ok = mbar_wait(a_full, 0, abort_flag, args.status, kTcTimeoutNs);
-            for (int t = 0; ok && t <= T; ++t) {
-                if (t < T) {
-                    const int s = t % NS, x = t & 1;
-                    ok = mbar_wait(&full[s], (t / NS) & 1, abort_flag, args.status, kTcTimeoutNs);
-                    if (ok && t >= 2) ok = mbar_wait(&s_free[x], ((t >> 1) - 1) & 1, abort_flag, args.status,
-                                                     kTcTimeoutNs);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sB = smem_u32(sm + L::Stage0 + s * L::kStage);
+            for (int t = 0; ok && t < T; ++t) {
+                const int x = t & 1;
+                ok = mbar_wait(&fullB[t % NB], (t / NB) & 1, abort_flag, args.status, kTcTimeoutNs);
+                // the buffer holds P(t - 2) until PV(t - 2) has completed
+                if (ok && t >= 2) ok = mbar_wait(&p_free[x], ((t - 2) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t b = dB + (uint64_t)(((t % NB) * L::kB) >> 4);
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t off = (k & 3) * 32;  // 16 elements = 32 bytes into the 128-byte row
-                        const uint64_t da = sdesc_sw128(sA + (k >> 2) * (BM * 128) + off, 16, 1024);
-                        const uint64_t db = sdesc_sw128(sB + (k >> 2) * (BN * 128) + off, 16, 1024);
-                        mma_f16_ss(tmem + x * BN, da, db, idS, k > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&s_full[x]);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    // 16 elements = 32 bytes into the 128-byte row; 64-element chunks stacked
+                    const uint64_t oa = (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
+                    const uint64_t ob = (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
+                    mma_f16_ss(tmem + x * BN, dA + oa, b + ob, idS, kk > 0 ? 1u : 0u);
                 }
-                if (t >= 1) {
-                    const int tp = t - 1, sp = tp % NS, xp = tp & 1;
-                    ok = mbar_wait(&p_full[xp], (tp >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sP = smem_u32(sm + L::P0 + xp * L::kP);
-                    const uint32_t sC = smem_u32(sm + L::Stage0 + sp * L::kStage + L::kB);
-#pragma unroll
-                    for (int k = 0; k < BN / 16; ++k) {
-                        const uint64_t da = sdesc_sw128(sP + k * 32, 16, 1024);
-                        const uint64_t db = sdesc_sw128(sC + k * (16 * 128), BN * 128, 1024);
-                        mma_f16_ss(tmem + 2 * BN, da, db, idO, (tp > 0 || k > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&p_free[xp]);
-                    mma_commit(&empty[sp]);
-                }
+                mma_commit(&s_full[x]);
+                mma_commit(&emptyB[t % NB]);
             }
-            // wind down: all issued MMAs complete before TMEM is released
-            mma_commit(drain);
+            mma_commit(&drain[0]);
             const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(drain, 0) && global_ns() - t0 < 1000000000ull) {
+            while (!mbar_try_wait(&drain[0], 0) && global_ns() - t0 < 1000000000ull) {
+            }
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ PV issuer: O += P(t) C_t
+        if (lane == 0 && T > 0) {
+            constexpr uint32_t idO = idesc_f16(BM, DV, 0, 0, 0, 1);   // f16 P (TMEM) x f16 C (MN-major)
+            const uint64_t dC = sdesc_sw128(smem_u32(sm + L::C0), BN * 128, 1024);
+            bool ok = true;
+            for (int t = 0; ok && t < T; ++t) {
+                const int x = t & 1;
+                ok = mbar_wait(&p_full[x], (t >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                if (ok) ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t c = dC + (uint64_t)(((t % NC) * L::kC) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_f16_ts(tO0, tmem + x * BN + 8 * kk, c + (uint64_t)((kk * 16 * 128) >> 4), idO,
+                               (t > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&p_free[x]);
+                mma_commit(&emptyC[t % NC]);
+            }
+            mma_commit(&drain[1]);
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(&drain[1], 0) && global_ns() - t0 < 1000000000ull) {
             }
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int q = warp & 3;
+        const int q = warp & 3;                 // TMEM lanes 32 q .. 32 q + 31
         const int row = q * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-        float m2 = -INFINITY, l = 0.f;
+        const uint32_t lanes = (uint32_t)(q * 32) << 16;
+        const uint32_t tO = tO0 + lanes;
+        const float cb = args.cb;
+        float m2 = -INFINITY, l = 0.f;          // running max (log2 units) and normaliser
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             const int x = t & 1;
+            const uint32_t tS = tmem + x * BN + lanes;
             ok = mbar_wait(&s_full[x], (t >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
             if (!ok) break;
             tc_fence_after();
-            float s[BN];
-            tmem_ld32(tl + x * BN, s);
-            tmem_ld32(tl + x * BN + 32, s + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[x]);
-
-            const int valid = min(BN, b_hi - (b_lo + t * BN));
-            float mt = -INFINITY;
+            const int valid = b_hi - (b_lo + t * BN);
+            // pass 1: row maximum over the 128 logits (two 64-column loads)
+            float mq[8];
 #pragma unroll
-            for (int j = 0; j < BN; ++j) {
-                s[j] = j < valid ? s[j] * args.cb : -INFINITY;
-                mt = fmaxf(mt, s[j]);
+            for (int i = 0; i < 8; ++i) mq[i] = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                tmem_ld64(tS + 64 * h, sv);
+                tmem_wait_ld();
+                if (valid < BN) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (64 * h + j >= valid) sv[j] = -INFINITY;
+                }
+#pragma unroll
+                for (int j = 0; j < 64; ++j) mq[j & 7] = fmaxf(mq[j & 7], sv[j]);
             }
+            const float mt = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                                   fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7]))) * cb;
             if (__any_sync(0xffffffffu, mt > m2 + kRescale)) {
                 const float mn = fmaxf(m2, mt);
                 if (t > 0) {
-                    // O holds tiles 0..t-1: wait for the last of them, then rescale in place
+                    // O holds key blocks 0..t-1: wait for the last of them, then rescale in place
                     ok = mbar_wait(&p_free[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
@@ -262,87 +298,101 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c0 = 0; c0 < DV; c0 += 32) {
                         float o[32];
-                        tmem_ld32(tl + 2 * BN + c0, o);
+                        tmem_ld32(tO + c0, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] *= sc;
-                        tmem_st32(tl + 2 * BN + c0, o);
+                        tmem_st32(tO + c0, o);
                     }
                     tmem_wait_st();
                     l *= sc;
                 }
                 m2 = mn;
             }
-            if (t >= 2) {
-                ok = mbar_wait(&p_free[x], ((t - 2) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+            if (MODE == kExpmmRownorm) {
+                // w arrives with the value tile; this stage cannot be reloaded before PV(t)
+                ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
             }
-            const float* wv = reinterpret_cast<const float*>(sm + L::Stage0 + (t % NS) * L::kStage + L::kB + L::kC);
-            unsigned char* prow = sm + L::P0 + x * L::kP + row * 128;
+            const float* wv = reinterpret_cast<const float*>(sm + L::Wv + (t % NC) * BN * 4);
+            const float nm = -m2;
+            float lp[4] = {0.f, 0.f, 0.f, 0.f};
+            // pass 2: P = 2^(S cb - m2) as fp16 pairs over the first 64 columns
 #pragma unroll
-            for (int c16 = 0; c16 < BN / 8; ++c16) {
-                uint32_t packed[4];
+            for (int h = 0; h < 2; ++h) {
+                float sv[64];
+                tmem_ld64(tS + 64 * h, sv);
+                tmem_wait_ld();
+                if (valid < BN) {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int j = c16 * 8 + 2 * h;
-                    const float p0 = ex2(s[j] - m2), p1 = ex2(s[j + 1] - m2);
-                    if (MODE == kExpmmRownorm)
-                        l += p0 * wv[j] + p1 * wv[j + 1];
-                    else
-                        l += p0 + p1;
-                    const __half2 hp = __floats2half2_rn(p0, p1);
-                    packed[h] = *reinterpret_cast<const uint32_t*>(&hp);
+                    for (int j = 0; j < 64; ++j)
+                        if (64 * h + j >= valid) sv[j] = -INFINITY;
                 }
-                *reinterpret_cast<uint4*>(prow + ((c16 ^ (row & 7)) << 4)) =
-                    make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                uint32_t packed[32];
+#pragma unroll
+                for (int j = 0; j < 64; j += 2) {
+                    const float p0 = ex2(fmaf(sv[j], cb, nm)), p1 = ex2(fmaf(sv[j + 1], cb, nm));
+                    if (MODE == kExpmmRownorm)
+                        lp[(j >> 1) & 3] = fmaf(p1, wv[64 * h + j + 1], fmaf(p0, wv[64 * h + j], lp[(j >> 1) & 3]));
+                    else
+                        lp[(j >> 1) & 3] += p0 + p1;
+                    const __half2 hp = __floats2half2_rn(p0, p1);
+                    packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                }
+                tmem_st32u(tS + 32 * h, packed);
             }
-            fence_async_smem();
+            l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[x]);
         }
 
-        // ------------------------------------------------------------ epilogue
-        float o[DV];
-#pragma unroll
-        for (int c = 0; c < DV; ++c) o[c] = 0.f;
+        // ------------------------------------------------------------ epilogue (32 columns at a time)
         if (ok && T > 0) {
             ok = mbar_wait(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
             ok = __all_sync(0xffffffffu, ok);
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int c0 = 0; c0 < DV; c0 += 32) tmem_ld32(tl + 2 * BN + c0, o + c0);
-                tmem_wait_ld();
-            }
+            if (ok) tc_fence_after();
         }
         const int a = a0 + row;
-        if (ok && a < a_valid) {
+        const bool store = ok && a < a_valid;
+        const bool have_o = ok && T > 0;
+        float* dst_p = static_cast<float*>(args.out) + (((size_t)unit * args.nsplit + split) * args.r + a) * (DV + 2);
+        float* dst_r = static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a) * DV;
+        const float* sg = args.sigma + (size_t)unit * DV;
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int c0 = 0; c0 < DV; c0 += 32) {
+            float o[32];
+            if (have_o) {
+                tmem_ld32(tO + c0, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = 0.f;
+            }
+            if (!store) continue;
             if (MODE == kExpmmPartial) {
-                float* dst = static_cast<float*>(args.out) +
-                             (((size_t)unit * args.nsplit + split) * args.r + a) * (DV + 2);
                 // rows are DV + 2 floats apart: 8-byte aligned, not 16
 #pragma unroll
-                for (int c = 0; c < DV; c += 2) *reinterpret_cast<float2*>(dst + c) = make_float2(o[c], o[c + 1]);
-                *reinterpret_cast<float2*>(dst + DV) = make_float2(l, m2 * kLn2);
+                for (int c = 0; c < 32; c += 2)
+                    *reinterpret_cast<float2*>(dst_p + c0 + c) = make_float2(o[c], o[c + 1]);
             } else {
-                float* dst = static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a) * DV;
-                const float* sg = args.sigma + (size_t)unit * DV;
-                const float inv = 1.f / l;
 #pragma unroll
-                for (int c = 0; c < DV; c += 4)
-                    *reinterpret_cast<float4*>(dst + c) =
-                        make_float4(o[c] * sg[c] * inv, o[c + 1] * sg[c + 1] * inv, o[c + 2] * sg[c + 2] * inv,
-                                    o[c + 3] * sg[c + 3] * inv);
+                for (int c = 0; c < 32; c += 4)
+                    *reinterpret_cast<float4*>(dst_r + c0 + c) =
+                        make_float4(o[c] * sg[c0 + c] * inv, o[c + 1] * sg[c0 + c + 1] * inv,
+                                    o[c + 2] * sg[c0 + c + 2] * inv, o[c + 3] * sg[c0 + c + 3] * inv);
             }
         }
+        if (MODE == kExpmmPartial && store) *reinterpret_cast<float2*>(dst_p + DV) = make_float2(l, m2 * kLn2);
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc<256>(tmem);
+    if (warp == 2) tmem_dealloc<512>(tmem);
 }
 
 // V (bf16) -> fp16 copy for the value operand of the weights GEMM.
@@ -454,7 +504,7 @@ wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K
     a.hq = s.hkv;
     a.group = 1;
     a.cb = (float)(s.beta * 1.4426950408889634);
-    dim3 grid((s.r + BM - 1) / BM, s.nsplit, s.units);
+    dim3 grid((s.r + TILES * BM - 1) / (TILES * BM), s.nsplit, s.units);
     return launch_tc<kExpmmPartial>(s.d, s.dv, mA, mB, mC, a, grid, st);
 }
 
@@ -487,7 +537,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     a.hq = s.hq;
     a.group = s.hq / s.hkv;
     a.cb = (float)(s.beta * 1.4426950408889634);
-    dim3 grid((s.nq + BM - 1) / BM, 1, s.batch * s.hq);
+    dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
     return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
 }
 
@@ -519,7 +569,7 @@ wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, con
     a.hq = s.hq;
     a.group = s.hq / s.hkv;
     a.cb = (float)(s.beta * 1.4426950408889634);
-    dim3 grid((s.nq + BM - 1) / BM, 1, s.batch * s.hq);
+    dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
     return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
 }
 
