@@ -11,11 +11,17 @@
 // normaliser column W[:, dv].  Weights: the (O, l, m) of each key split are
 // written for the solve; attention: out = O sigma / l.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads (A once, then B, C and w
-// tiles through a 3-stage ring), warp 1 owns TMEM and issues the MMAs, warps
-// 2..5 run the exponentials and the epilogue (warp w reads TMEM lanes
-// 32 (w % 4) .. +31, one tile row per thread).  S is double buffered in
-// TMEM (2 x 64 columns), O takes DV columns.  Operands use the 128-byte
+// Warp roles (384 threads): warp 0 loads A once and then the key tiles, warp 1
+// the value tiles (TMA, 3-stage rings); warp 2 owns TMEM and issues S = A B^T,
+// warp 3 issues O += P C; warps 4..11 run the exponentials and the epilogue.
+// A softmax warp w reads TMEM lanes 32 (w % 4) .. +31 (one tile row per
+// thread) and takes every other key tile (parity (w - 4) / 4), so the two
+// warps on an SM sub-partition alternate: one loads S and finds its row
+// maxima while the other runs its exponentials.  They share one reference
+// maximum per row (the shift of O), handed from tile to tile through shared
+// memory at named barriers; O is rescaled only when the reference grows by
+// more than 2^8.  S is triple buffered in TMEM (3 x 128 columns), O takes
+// the remaining DV columns.  Operands use the 128-byte
 // swizzled canonical layouts: A, B and P K-major, C MN-major.  Every wait is
 // bounded; a wait that runs out records WC_ERR_TIMEOUT and the block winds
 // down (drains its copies and MMAs, frees TMEM) instead of hanging.
@@ -38,8 +44,16 @@ constexpr int TILES = 1;             // row tiles per CTA
 constexpr int BN = 128;              // keys per stage
 constexpr int NB = 3;                // key-tile stages: released once S is computed
 constexpr int NC = 3;                // value-tile stages: released once PV is computed
-// warps: 0 key loader, 1 value loader, 2 S issuer, 3 PV issuer, 4..7 softmax
-constexpr int kThreads = 256;
+// warps: 0 key loader, 1 value loader, 2 S issuer, 3 PV issuer, 4..11 softmax
+constexpr int kThreads = 384;
+constexpr int NS = 3;                // S / P buffers in TMEM
+// Register split (setmaxnreg): the block is launched with kRegsLaunch per
+// thread; warps 0..3 drop to kRegsSide and warps 4..11 rise to kRegsSoftmax,
+// which together use exactly the launch's registers (checked on the host).
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsSide = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // log2 units: P stays below 2^8 between rescales
 constexpr uint64_t kTcTimeoutNs = 4000000000ull;
@@ -68,31 +82,37 @@ struct Smem {
     static constexpr uint32_t B0 = kA;                  // [NB] key tiles
     static constexpr uint32_t C0 = B0 + NB * kB;        // [NC] value tiles
     static constexpr uint32_t Wv = C0 + NC * kC;        // [NC][BN] normaliser weights (rownorm)
-    static constexpr uint32_t Bar = Wv + NC * BN * 4;
+    static constexpr uint32_t Tok = Wv + NC * BN * 4;   // [2][BM] fp32: reference maxima, then sums
+    static constexpr uint32_t Bar = Tok + 2 * BM * 4;
     static constexpr uint32_t kTotal = Bar + 256;
-    static constexpr uint32_t kAlloc = kTotal + 1024;   // room to align the base to 1024
+    static constexpr uint32_t kAlloc = kTotal;          // the base is 1024-aligned (checked in the kernel)
+    static_assert(kAlloc <= 232448, "shared memory per block");
 };
 
-// TMEM: S / P buffer x (x = key block & 1) at columns 128 x .. +127 (P as fp16
-// pairs over the first 64 columns of the S it came from), O at 256 .. 256+DV-1.
+// TMEM: S / P buffer b (b = key block % 3) at columns 128 b .. +127 (P as
+// fp16 pairs over the first 64 columns of the S it came from), O at
+// 384 .. 384+DV-1.
 template <int D, int DV, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     expmm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                     const __grid_constant__ CUtensorMap mapC, const TcArgs args) {
     using L = Smem<D, DV>;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw;
+    if (smem_u32(sm) & 1023u) {  // the swizzled tiles need 1024-byte alignment
+        if (threadIdx.x == 0) record_status(args.status, WC_ERR_UNSUPPORTED);
+        return;
+    }
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::Bar);
     uint64_t* fullB = bars;                   // [NB]
     uint64_t* emptyB = fullB + NB;            // [NB]
     uint64_t* fullC = emptyB + NB;            // [NC]
     uint64_t* emptyC = fullC + NC;            // [NC]
     uint64_t* a_full = emptyC + NC;
-    uint64_t* s_full = a_full + 1;            // [2]
-    uint64_t* p_full = s_full + 2;            // [2]
-    uint64_t* p_free = p_full + 2;            // [2]
-    uint64_t* drain = p_free + 2;             // [2] (S issuer, PV issuer)
+    uint64_t* s_full = a_full + 1;            // [NS]
+    uint64_t* p_full = s_full + NS;           // [NS]
+    uint64_t* p_free = p_full + NS;           // [NS]
+    uint64_t* drain = p_free + NS;            // [2] (S issuer, PV issuer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -129,12 +149,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&emptyC[i], 1);
         }
         mbar_init(a_full, 1);
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < NS; ++x) {
             mbar_init(&s_full[x], 1);
             mbar_init(&p_full[x], 4);
             mbar_init(&p_free[x], 1);
-            mbar_init(&drain[x], 1);
         }
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -143,227 +164,286 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tO0 = tmem + 2 * BN;
+    const uint32_t tO0 = tmem + NS * BN;
 
-    if (warp <= 1) {
-        // ------------------------------------------------------------ TMA producers
-        // warp 0 loads A once, then the key tiles; warp 1 the value tiles (and w)
-        const bool keys = warp == 0;
-        if (lane == 0 && T > 0) {
-            if (keys) {
-                tma_prefetch(&mapA);
-                tma_prefetch(&mapB);
-                mbar_expect_tx(a_full, L::kA);
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) tma_load_2d(sm + L::A + c * (BM * 128), &mapA, a_full, c * 64, a_row0);
-            } else {
-                tma_prefetch(&mapC);
-            }
-            const int NR = keys ? NB : NC;
-            uint64_t* fl = keys ? fullB : fullC;
-            uint64_t* em = keys ? emptyB : emptyC;
-            int issued = 0;
-            for (int t = 0; t < T; ++t) {
-                const int s = t % NR;
-                if (t >= NR && !mbar_wait(&em[s], ((t / NR) - 1) & 1, abort_flag, args.status, kTcTimeoutNs))
-                    break;
-                const int brow = b_row0 + t * BN;
+    if (warp < 4) {
+        reg_release<kRegsSide>();             // loaders and issuers: few registers
+        if (warp <= 1) {
+            // ------------------------------------------------------------ TMA producers
+            // warp 0 loads A once, then the key tiles; warp 1 the value tiles (and w)
+            const bool keys = warp == 0;
+            if (lane == 0 && T > 0) {
                 if (keys) {
-                    mbar_expect_tx(&fl[s], L::kB);
-                    unsigned char* st = sm + L::B0 + s * L::kB;
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &fl[s], c * 64, brow);
+                    tma_prefetch(&mapA);
+                    tma_prefetch(&mapB);
+                    mbar_expect_tx(a_full, L::kA);
+    #pragma unroll
+                    for (int c = 0; c < D / 64; ++c) tma_load_2d(sm + L::A + c * (BM * 128), &mapA, a_full, c * 64, a_row0);
                 } else {
-                    mbar_expect_tx(&fl[s], L::kC + (MODE == kExpmmRownorm ? BN * 4 : 0));
-                    unsigned char* st = sm + L::C0 + s * L::kC;
-#pragma unroll
-                    for (int c = 0; c < DV / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapC, &fl[s], c * 64, brow);
-                    if (MODE == kExpmmRownorm)
-                        bulk_load(sm + L::Wv + s * BN * 4, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN,
-                                  BN * 4, &fl[s]);
+                    tma_prefetch(&mapC);
                 }
-                issued = t + 1;
-            }
-            // wind down: every copy this thread started has landed before the block exits
-            if (*abort_flag) {
-                const uint64_t t0 = global_ns();
-                while (keys && !mbar_try_wait(a_full, 0) && global_ns() - t0 < 100000000ull) {
+                const int NR = keys ? NB : NC;
+                uint64_t* fl = keys ? fullB : fullC;
+                uint64_t* em = keys ? emptyB : emptyC;
+                int issued = 0;
+                for (int t = 0; t < T; ++t) {
+                    const int s = t % NR;
+                    if (t >= NR && !mbar_wait(&em[s], ((t / NR) - 1) & 1, abort_flag, args.status, kTcTimeoutNs))
+                        break;
+                    const int brow = b_row0 + t * BN;
+                    if (keys) {
+                        mbar_expect_tx(&fl[s], L::kB);
+                        unsigned char* st = sm + L::B0 + s * L::kB;
+    #pragma unroll
+                        for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &fl[s], c * 64, brow);
+                    } else {
+                        mbar_expect_tx(&fl[s], L::kC + (MODE == kExpmmRownorm ? BN * 4 : 0));
+                        unsigned char* st = sm + L::C0 + s * L::kC;
+    #pragma unroll
+                        for (int c = 0; c < DV / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapC, &fl[s], c * 64, brow);
+                        if (MODE == kExpmmRownorm)
+                            bulk_load(sm + L::Wv + s * BN * 4, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN,
+                                      BN * 4, &fl[s]);
+                    }
+                    issued = t + 1;
                 }
-                for (int t = issued - NR > 0 ? issued - NR : 0; t < issued; ++t) {
-                    const uint64_t t1 = global_ns();
-                    while (!mbar_try_wait(&fl[t % NR], (t / NR) & 1) && global_ns() - t1 < 100000000ull) {
+                // wind down: every copy this thread started has landed before the block exits
+                if (*abort_flag) {
+                    const uint64_t t0 = global_ns();
+                    while (keys && !mbar_try_wait(a_full, 0) && global_ns() - t0 < 100000000ull) {
+                    }
+                    for (int t = issued - NR > 0 ? issued - NR : 0; t < issued; ++t) {
+                        const uint64_t t1 = global_ns();
+                        while (!mbar_try_wait(&fl[t % NR], (t / NR) & 1) && global_ns() - t1 < 100000000ull) {
+                        }
                     }
                 }
             }
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ S issuer: S(t) = A B_t^T into buffer t & 1
-        if (lane == 0 && T > 0) {
-            constexpr uint32_t idS = idesc_f16(BM, BN, 1, 1, 0, 0);   // bf16 x bf16, both K-major
-            const uint64_t dA = sdesc_sw128(smem_u32(sm + L::A), 16, 1024);
-            const uint64_t dB = sdesc_sw128(smem_u32(sm + L::B0), 16, 1024);
-            bool ok = mbar_wait(a_full, 0, abort_flag, args.status, kTcTimeoutNs);
-            for (int t = 0; ok && t < T; ++t) {
-                const int x = t & 1;
-                ok = mbar_wait(&fullB[t % NB], (t / NB) & 1, abort_flag, args.status, kTcTimeoutNs);
-                // the buffer holds P(t - 2) until PV(t - 2) has completed
-                if (ok && t >= 2) ok = mbar_wait(&p_free[x], ((t - 2) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
-                if (!ok) break;
-                tc_fence_after();
-                const uint64_t b = dB + (uint64_t)(((t % NB) * L::kB) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    // 16 elements = 32 bytes into the 128-byte row; 64-element chunks stacked
-                    const uint64_t oa = (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
-                    const uint64_t ob = (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
-                    mma_f16_ss(tmem + x * BN, dA + oa, b + ob, idS, kk > 0 ? 1u : 0u);
+        } else if (warp == 2) {
+            // ------------------------------------------------------------ S issuer: S(t) = A B_t^T into buffer t % NS
+            if (lane == 0 && T > 0) {
+                constexpr uint32_t idS = idesc_f16(BM, BN, 1, 1, 0, 0);   // bf16 x bf16, both K-major
+                const uint64_t dA = sdesc_sw128(smem_u32(sm + L::A), 16, 1024);
+                const uint64_t dB = sdesc_sw128(smem_u32(sm + L::B0), 16, 1024);
+                bool ok = mbar_wait(a_full, 0, abort_flag, args.status, kTcTimeoutNs);
+                for (int t = 0; ok && t < T; ++t) {
+                    const int x = t % NS;
+                    ok = mbar_wait(&fullB[t % NB], (t / NB) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    // the buffer holds P(t - NS) until PV(t - NS) has completed
+                    if (ok && t >= NS) ok = mbar_wait(&p_free[x], ((t / NS) - 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t b = dB + (uint64_t)(((t % NB) * L::kB) >> 4);
+    #pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        // 16 elements = 32 bytes into the 128-byte row; 64-element chunks stacked
+                        const uint64_t oa = (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
+                        const uint64_t ob = (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
+                        mma_f16_ss(tmem + x * BN, dA + oa, b + ob, idS, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[x]);
+                    mma_commit(&emptyB[t % NB]);
                 }
-                mma_commit(&s_full[x]);
-                mma_commit(&emptyB[t % NB]);
+                mma_commit(&drain[0]);
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(&drain[0], 0) && global_ns() - t0 < 1000000000ull) {
+                }
             }
-            mma_commit(&drain[0]);
-            const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&drain[0], 0) && global_ns() - t0 < 1000000000ull) {
-            }
-        }
-    } else if (warp == 3) {
-        // ------------------------------------------------------------ PV issuer: O += P(t) C_t
-        if (lane == 0 && T > 0) {
-            constexpr uint32_t idO = idesc_f16(BM, DV, 0, 0, 0, 1);   // f16 P (TMEM) x f16 C (MN-major)
-            const uint64_t dC = sdesc_sw128(smem_u32(sm + L::C0), BN * 128, 1024);
-            bool ok = true;
-            for (int t = 0; ok && t < T; ++t) {
-                const int x = t & 1;
-                ok = mbar_wait(&p_full[x], (t >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
-                if (ok) ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
-                if (!ok) break;
-                tc_fence_after();
-                const uint64_t c = dC + (uint64_t)(((t % NC) * L::kC) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_f16_ts(tO0, tmem + x * BN + 8 * kk, c + (uint64_t)((kk * 16 * 128) >> 4), idO,
-                               (t > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&p_free[x]);
-                mma_commit(&emptyC[t % NC]);
-            }
-            mma_commit(&drain[1]);
-            const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&drain[1], 0) && global_ns() - t0 < 1000000000ull) {
+        } else if (warp == 3) {
+            // ------------------------------------------------------------ PV issuer: O += P(t) C_t
+            if (lane == 0 && T > 0) {
+                constexpr uint32_t idO = idesc_f16(BM, DV, 0, 0, 0, 1);   // f16 P (TMEM) x f16 C (MN-major)
+                const uint64_t dC = sdesc_sw128(smem_u32(sm + L::C0), BN * 128, 1024);
+                bool ok = true;
+                for (int t = 0; ok && t < T; ++t) {
+                    const int x = t % NS;
+                    ok = mbar_wait(&p_full[x], (t / NS) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (ok) ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t c = dC + (uint64_t)(((t % NC) * L::kC) >> 4);
+    #pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_f16_ts(tO0, tmem + x * BN + 8 * kk, c + (uint64_t)((kk * 16 * 128) >> 4), idO,
+                                   (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&p_free[x]);
+                    mma_commit(&emptyC[t % NC]);
+                }
+                mma_commit(&drain[1]);
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(&drain[1], 0) && global_ns() - t0 < 1000000000ull) {
+                }
             }
         }
     } else {
+        reg_claim<kRegsSoftmax>();            // softmax warps: a whole S row per thread
         // ------------------------------------------------------------ softmax + epilogue
         const int q = warp & 3;                 // TMEM lanes 32 q .. 32 q + 31
+        const int par = (warp - 4) >> 2;        // this warp takes the key tiles t with t % 2 == par
         const int row = q * 32 + lane;
+        // named barriers that hand the reference on: 1 + q from parity 0 to 1, 5 + q back
+        const int id_in = par ? 1 + q : 5 + q;
+        const int id_out = par ? 5 + q : 1 + q;
         const uint32_t lanes = (uint32_t)(q * 32) << 16;
-        const uint32_t tO = tO0 + lanes;
+        float* tok = reinterpret_cast<float*>(sm + L::Tok);   // [2][BM]
         const float cb = args.cb;
-        float m2 = -INFINITY, l = 0.f;          // running max (log2 units) and normaliser
+        float mO = -INFINITY;                   // the reference of O (log2 units) as this warp knows it
+        float l = 0.f;                          // this warp's share of the normaliser, relative to mO
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int x = t & 1;
+        // Every iteration runs the same barrier steps whatever `ok` is, so a warp
+        // that gave up still hands the reference on and its partner never hangs.
+        for (int t = par; t < T; t += 2) {
+            const int x = t % NS;
             const uint32_t tS = tmem + x * BN + lanes;
-            ok = mbar_wait(&s_full[x], (t >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
-            if (!ok) break;
-            tc_fence_after();
+            ok = ok && mbar_wait(&s_full[x], (t / NS) & 1, abort_flag, args.status, kTcTimeoutNs);
+            ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
             const int valid = b_hi - (b_lo + t * BN);
-            // pass 1: row maximum over the 128 logits (two 64-column loads)
-            float mq[8];
+            // pass 1: the whole row of S into registers, and its maximum
+            float sv[BN];
+            float mt = -INFINITY;
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mq[i] = -INFINITY;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float sv[64];
-                tmem_ld64(tS + 64 * h, sv);
+                for (int h = 0; h < 4; ++h) tmem_ld32(tS + 32 * h, sv + 32 * h);
                 tmem_wait_ld();
                 if (valid < BN) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (64 * h + j >= valid) sv[j] = -INFINITY;
+                    for (int j = 0; j < BN; ++j)
+                        if (j >= valid) sv[j] = -INFINITY;
                 }
+                float mq[8];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) mq[j & 7] = fmaxf(mq[j & 7], sv[j]);
+                for (int i = 0; i < 8; ++i) mq[i] = sv[i];
+#pragma unroll
+                for (int j = 8; j < BN; ++j) mq[j & 7] = fmaxf(mq[j & 7], sv[j]);
+                mt = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                           fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7]))) * cb;
             }
-            const float mt = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
-                                   fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7]))) * cb;
-            if (__any_sync(0xffffffffu, mt > m2 + kRescale)) {
-                const float mn = fmaxf(m2, mt);
-                if (t > 0) {
-                    // O holds key blocks 0..t-1: wait for the last of them, then rescale in place
-                    ok = mbar_wait(&p_free[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const float sc = (m2 == -INFINITY) ? 0.f : ex2(m2 - mn);
-#pragma unroll
-                    for (int c0 = 0; c0 < DV; c0 += 32) {
-                        float o[32];
-                        tmem_ld32(tO + c0, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= sc;
-                        tmem_st32(tO + c0, o);
-                    }
-                    tmem_wait_st();
-                    l *= sc;
+            // the reference after tile t - 1 (decided by the partner)
+            if (t > 0) {
+                pair_sync(id_in);
+                const float mp = tok[row];
+                if (mp != mO) {
+                    if (mO != -INFINITY) l *= ex2(mO - mp);
+                    mO = mp;
                 }
-                m2 = mn;
             }
-            if (MODE == kExpmmRownorm) {
+            const bool grow = __any_sync(0xffffffffu, ok && mt > mO + kRescale);
+            const float mn = grow ? fmaxf(mO, mt) : mO;
+            const float mold = mO;
+            if (grow) {
+                if (mO != -INFINITY) l *= ex2(mO - mn);
+                mO = mn;
+            }
+            if (t + 1 < T) tok[row] = mn;       // the partner reads it after this tile's hand-over below
+            if (ok && MODE == kExpmmRownorm) {
                 // w arrives with the value tile; this stage cannot be reloaded before PV(t)
                 ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
                 ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
             }
-            const float* wv = reinterpret_cast<const float*>(sm + L::Wv + (t % NC) * BN * 4);
-            const float nm = -m2;
-            float lp[4] = {0.f, 0.f, 0.f, 0.f};
-            // pass 2: P = 2^(S cb - m2) as fp16 pairs over the first 64 columns
+            if (ok) {
+                // pass 2: P = 2^(S cb - mO) as fp16 pairs over the first 64 columns
+                const float* wv = reinterpret_cast<const float*>(sm + L::Wv + (t % NC) * BN * 4);
+                const float nm = -mO;
+                float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float sv[64];
-                tmem_ld64(tS + 64 * h, sv);
-                tmem_wait_ld();
-                if (valid < BN) {
+                for (int h = 0; h < 4; ++h) {
+                    const float* sh = sv + 32 * h;
+                    uint32_t packed[16];
+                    float w[MODE == kExpmmRownorm ? 32 : 1];
+                    if (MODE == kExpmmRownorm) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (64 * h + j >= valid) sv[j] = -INFINITY;
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 f = lds_f4_ordered(wv + 32 * h + j);
+                            w[j] = f.x;
+                            w[j + 1] = f.y;
+                            w[j + 2] = f.z;
+                            w[j + 3] = f.w;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const float p0 = ex2_ordered(fmaf(sh[j], cb, nm)), p1 = ex2_ordered(fmaf(sh[j + 1], cb, nm));
+                        if (MODE == kExpmmRownorm)
+                            lp[(j >> 1) & 3] = fmaf(p1, w[j + 1], fmaf(p0, w[j], lp[(j >> 1) & 3]));
+                        else
+                            lp[(j >> 1) & 3] += p0 + p1;
+                        const __half2 hp = __floats2half2_rn(p0, p1);
+                        packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                    }
+                    tmem_st16u(tS + 16 * h, packed);
                 }
-                uint32_t packed[32];
+                l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+                tmem_wait_st();
+                if (grow && t > 0) {
+                    // O holds key blocks 0..t-1 in the old reference: once the last of them
+                    // has landed, rescale it in place (PV(t) is issued only after this)
+                    ok = mbar_wait(&p_free[(t - 1) % NS], ((t - 1) / NS) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (ok) {
+                        tc_fence_after();
+                        const float sc = (mold == -INFINITY) ? 0.f : ex2(mold - mn);
 #pragma unroll
-                for (int j = 0; j < 64; j += 2) {
-                    const float p0 = ex2(fmaf(sv[j], cb, nm)), p1 = ex2(fmaf(sv[j + 1], cb, nm));
-                    if (MODE == kExpmmRownorm)
-                        lp[(j >> 1) & 3] = fmaf(p1, wv[64 * h + j + 1], fmaf(p0, wv[64 * h + j], lp[(j >> 1) & 3]));
-                    else
-                        lp[(j >> 1) & 3] += p0 + p1;
-                    const __half2 hp = __floats2half2_rn(p0, p1);
-                    packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                        for (int c0 = 0; c0 < DV; c0 += 32) {
+                            float o[32];
+                            tmem_ld32(tO0 + lanes + c0, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] *= sc;
+                            tmem_st32(tO0 + lanes + c0, o);
+                        }
+                        tmem_wait_st();
+                    }
                 }
-                tmem_st32u(tS + 32 * h, packed);
+                if (ok) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_full[x]);
+                }
             }
-            l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[x]);
+            // hand the reference on once this tile's exponentials are done, so the two
+            // warps of the sub-partition take turns on the exponential unit
+            if (t + 1 < T) pair_arrive(id_out);
         }
 
-        // ------------------------------------------------------------ epilogue (32 columns at a time)
+        // ------------------------------------------------------------ epilogue
+        // The warp that took the last tile (parity (T - 1) & 1; parity 1 when
+        // T == 0) knows the final reference.  The other hands it log2 of its
+        // share of the normaliser in its own reference; the last one adds the
+        // two in the final reference and hands the total back.
+        const bool last = par == ((T + 1) & 1);
+        float* tl = tok + BM;                   // second slot: only the epilogue uses it
+        float lt;
+        // (its own barrier 9 + q first: its last hand-over may not have been taken yet)
+        if (!last) {
+            tl[row] = (l > 0.f) ? __log2f(l) + mO : -INFINITY;
+            pair_arrive(9 + q);
+            pair_sync(id_in);
+            lt = tl[row];
+        } else {
+            pair_sync(9 + q);
+            const float lo = tl[row];
+            lt = l + ((lo == -INFINITY) ? 0.f : ex2(lo - mO));
+            tl[row] = lt;
+            pair_arrive(id_out);
+        }
         if (ok && T > 0) {
-            ok = mbar_wait(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+            ok = mbar_wait(&p_free[(T - 1) % NS], ((T - 1) / NS) & 1, abort_flag, args.status, kTcTimeoutNs);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) tc_fence_after();
         }
+        // each warp writes half of O's columns
         const int a = a0 + row;
         const bool store = ok && a < a_valid;
         const bool have_o = ok && T > 0;
+        const uint32_t tO = tO0 + lanes + par * (DV / 2);
+        const int cbase = par * (DV / 2);
         float* dst_p = static_cast<float*>(args.out) + (((size_t)unit * args.nsplit + split) * args.r + a) * (DV + 2);
         float* dst_r = static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a) * DV;
         const float* sg = args.sigma + (size_t)unit * DV;
-        const float inv = 1.f / l;
+        const float inv = 1.f / lt;
 #pragma unroll
-        for (int c0 = 0; c0 < DV; c0 += 32) {
+        for (int c0 = 0; c0 < DV / 2; c0 += 32) {
             float o[32];
             if (have_o) {
                 tmem_ld32(tO + c0, o);
@@ -372,21 +452,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0.f;
             }
-            if (!store) continue;
-            if (MODE == kExpmmPartial) {
-                // rows are DV + 2 floats apart: 8-byte aligned, not 16
+            if (store) {
+                if (MODE == kExpmmPartial) {
+                    // rows are DV + 2 floats apart: 8-byte aligned, not 16
 #pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    *reinterpret_cast<float2*>(dst_p + c0 + c) = make_float2(o[c], o[c + 1]);
-            } else {
+                    for (int c = 0; c < 32; c += 2)
+                        *reinterpret_cast<float2*>(dst_p + cbase + c0 + c) = make_float2(o[c], o[c + 1]);
+                } else {
 #pragma unroll
-                for (int c = 0; c < 32; c += 4)
-                    *reinterpret_cast<float4*>(dst_r + c0 + c) =
-                        make_float4(o[c] * sg[c0 + c] * inv, o[c + 1] * sg[c0 + c + 1] * inv,
-                                    o[c + 2] * sg[c0 + c + 2] * inv, o[c + 3] * sg[c0 + c + 3] * inv);
+                    for (int c = 0; c < 32; c += 4) {
+                        const int cc = cbase + c0 + c;
+                        *reinterpret_cast<float4*>(dst_r + cc) =
+                            make_float4(o[c] * sg[cc] * inv, o[c + 1] * sg[cc + 1] * inv,
+                                        o[c + 2] * sg[cc + 2] * inv, o[c + 3] * sg[cc + 3] * inv);
+                    }
+                }
             }
         }
-        if (MODE == kExpmmPartial && store) *reinterpret_cast<float2*>(dst_p + DV) = make_float2(l, m2 * kLn2);
+        if (MODE == kExpmmPartial && store && last) *reinterpret_cast<float2*>(dst_p + DV) = make_float2(lt, mO * kLn2);
     }
 
     tc_fence_before();
@@ -458,6 +541,10 @@ wc_status launch_tc_t(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
     auto kern = expmm_tc_kernel<D, DV, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc) != cudaSuccess)
         return WC_ERR_CUDA;
+    // the register split needs the block launched with kRegsLaunch registers a thread
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return WC_ERR_CUDA;
+    if (fa.numRegs < kRegsLaunch) return WC_ERR_UNSUPPORTED;
     kern<<<grid, kThreads, L::kAlloc, st>>>(A, B, C, a);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
