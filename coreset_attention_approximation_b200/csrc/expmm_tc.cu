@@ -341,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
                 ok = __all_sync(0xffffffffu, ok);
             }
+            bool handed = false;
             if (ok) {
                 // pass 2: P = 2^(S cb - mO) as fp16 pairs over the first 64 columns
                 const float* wv = reinterpret_cast<const float*>(sm + L::Wv + (t % NC) * BN * 4);
@@ -348,6 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
+                    if (h == 3) {
+                        // hand the reference on before the last quarter: the partner's
+                        // exponentials start as this warp's drain from the unit
+                        if (t + 1 < T) pair_arrive(id_out);
+                        handed = true;
+                    }
                     const float* sh = sv + 32 * h;
                     uint32_t packed[16];
                     float w[MODE == kExpmmRownorm ? 32 : 1];
@@ -401,9 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) mbar_arrive(&p_full[x]);
                 }
             }
-            // hand the reference on once this tile's exponentials are done, so the two
-            // warps of the sub-partition take turns on the exponential unit
-            if (t + 1 < T) pair_arrive(id_out);
+            // (if pass 2 was skipped, hand the reference on here: the partner never hangs)
+            if (!handed && t + 1 < T) pair_arrive(id_out);
         }
 
         // ------------------------------------------------------------ epilogue
