@@ -87,6 +87,7 @@ struct Smem {
     static constexpr uint32_t kTotal = Bar + 256;
     static constexpr uint32_t kAlloc = kTotal;          // the base is 1024-aligned (checked in the kernel)
     static_assert(kAlloc <= 232448, "shared memory per block");
+    static_assert(BM * (DV + 4) * 4 <= NC * kC, "the epilogue stages O in the value ring");
 };
 
 // TMEM: S / P buffer b (b = key block % 3) at columns 128 b .. +127 (P as
@@ -438,16 +439,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (ok) tc_fence_after();
         }
-        // each warp writes half of O's columns
-        const int a = a0 + row;
-        const bool store = ok && a < a_valid;
+        // O goes out through shared memory (the value ring is idle once PV(T - 1)
+        // has completed): each warp stages half of the columns of its 32 rows,
+        // then the 256 softmax threads copy the block's rows, which are
+        // contiguous in global memory, with coalesced stores.
+        constexpr int SST = (MODE == kExpmmPartial) ? DV + 2 : DV + 4;   // staged row stride (floats)
+        float* stg = reinterpret_cast<float*>(sm + L::C0);
         const bool have_o = ok && T > 0;
         const uint32_t tO = tO0 + lanes + par * (DV / 2);
         const int cbase = par * (DV / 2);
-        float* dst_p = static_cast<float*>(args.out) + (((size_t)unit * args.nsplit + split) * args.r + a) * (DV + 2);
-        float* dst_r = static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a) * DV;
         const float* sg = args.sigma + (size_t)unit * DV;
         const float inv = 1.f / lt;
+        float* srow = stg + row * SST + cbase;
 #pragma unroll
         for (int c0 = 0; c0 < DV / 2; c0 += 32) {
             float o[32];
@@ -458,24 +461,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0.f;
             }
-            if (store) {
-                if (MODE == kExpmmPartial) {
-                    // rows are DV + 2 floats apart: 8-byte aligned, not 16
+            if (MODE == kExpmmPartial) {
+                // staged rows are DV + 2 floats apart (the global layout): 8-byte aligned
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2)
-                        *reinterpret_cast<float2*>(dst_p + cbase + c0 + c) = make_float2(o[c], o[c + 1]);
-                } else {
+                for (int c = 0; c < 32; c += 2)
+                    *reinterpret_cast<float2*>(srow + c0 + c) = make_float2(o[c], o[c + 1]);
+            } else {
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4) {
-                        const int cc = cbase + c0 + c;
-                        *reinterpret_cast<float4*>(dst_r + cc) =
-                            make_float4(o[c] * sg[cc] * inv, o[c + 1] * sg[cc + 1] * inv,
-                                        o[c + 2] * sg[cc + 2] * inv, o[c + 3] * sg[cc + 3] * inv);
-                    }
+                for (int c = 0; c < 32; c += 4) {
+                    const int cc = cbase + c0 + c;
+                    *reinterpret_cast<float4*>(srow + c0 + c) =
+                        make_float4(o[c] * sg[cc] * inv, o[c + 1] * sg[cc + 1] * inv, o[c + 2] * sg[cc + 2] * inv,
+                                    o[c + 3] * sg[cc + 3] * inv);
                 }
             }
         }
-        if (MODE == kExpmmPartial && store && last) *reinterpret_cast<float2*>(dst_p + DV) = make_float2(lt, mO * kLn2);
+        if (MODE == kExpmmPartial && last) *reinterpret_cast<float2*>(stg + row * SST + DV) = make_float2(lt, mO * kLn2);
+        softmax_sync();                         // all 8 softmax warps have staged their part
+        const int rows = min(BM, a_valid - a0);
+        const int st = tid - 4 * 32;            // 0 .. 255
+        if (ok) {
+            if (MODE == kExpmmPartial) {
+                // rows a0 .. of this split are one contiguous run of rows * (DV + 2) floats
+                float2* dst = reinterpret_cast<float2*>(static_cast<float*>(args.out) +
+                                                        (((size_t)unit * args.nsplit + split) * args.r + a0) * (DV + 2));
+                const float2* src = reinterpret_cast<const float2*>(stg);
+                const int n2 = rows * (DV + 2) / 2;
+                for (int i = st; i < n2; i += 256) dst[i] = src[i];
+            } else {
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a0) * DV);
+                const int n4 = rows * (DV / 4);
+                for (int i = st; i < n4; i += 256) {
+                    const int rr = i / (DV / 4), c4 = i - rr * (DV / 4);
+                    dst[i] = *reinterpret_cast<const float4*>(stg + rr * SST + 4 * c4);
+                }
+            }
+        }
     }
 
     tc_fence_before();

@@ -299,6 +299,8 @@ __device__ __forceinline__ bool pair_sync_and(int id, bool v) {
 }
 
 __device__ __forceinline__ void pair_sync(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+// Named barrier 13 over the 8 softmax warps (256 threads).
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 13, 256;" ::: "memory"); }
 __device__ __forceinline__ void pair_arrive(int id) { asm volatile("bar.arrive %0, 64;" ::"r"(id) : "memory"); }
 
 // ex2 kept in program order with the TMEM stores around it, so a long run of
