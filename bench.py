@@ -36,9 +36,11 @@ from coreset_attention_approximation_b200.workloads import WORKLOADS, make_input
 METRIC = "WildCat forward tokens/sec at 1 B200; select HBM GB/s and GEMM TC-util vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# dram bytes (read + write) per select launch per unit from an ncu capture of
-# the current select kernel (scaled by units); None until one is taken.
-SELECT_DRAM_BYTES_PER_UNIT = None
+# dram bytes (read + write) per select launch per unit, from a one-pass ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current select
+# kernel on the named workload: long = 9.475972 TB + 8.898401 GB over 8 units
+# (profiles/select_rpcholesky_long8.md).  Other workloads: not captured.
+SELECT_DRAM_BYTES_PER_UNIT = {"long": (9.475972e12 + 8.898401e9) / 8}
 
 
 def load_peaks():
@@ -313,7 +315,7 @@ def run_ours(args, world, rank, local):
     achieved = sb / (sel_avg * 1e-3) / 1e9
     f1, f2 = gemm_flops(w)
     wts_avg, att_avg = sum(wts_ms) / len(wts_ms), sum(att_ms) / len(att_ms)
-    traffic = None if SELECT_DRAM_BYTES_PER_UNIT is None else SELECT_DRAM_BYTES_PER_UNIT * w.batch * w.hkv
+    traffic = SELECT_DRAM_BYTES_PER_UNIT[w.name] * w.batch * w.hkv if w.name in SELECT_DRAM_BYTES_PER_UNIT else None
     tokens = w.batch * w.n_q * world
     res = {
         "metric": METRIC,
@@ -378,7 +380,7 @@ def kernel_breakdown(step):
             short = ("weights_gemm", "attend_gemm")[int(m.group(2))]
         else:
             for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
-                             ("merge_c1", "merge_c1"), ("trsv_kernel", "solve"), ("weights_prep", "w_prep")):
+                             ("merge_c1", "merge_c1"), ("trsm_kernel", "solve"), ("weights_prep", "w_prep")):
                 if key in name:
                     short = tag
                     break

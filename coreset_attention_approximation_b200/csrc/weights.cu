@@ -5,7 +5,7 @@
 // compressed as V_S = W V.  Here the weights act on [V | 1], so the softmax
 // normaliser is compressed with the values:
 //   C1 = exp(beta K_S K^T) [V | 1]           (gather + exp-GEMM, split over keys)
-//   W  = L^-T (L^-1 C1),  L = F[piv, :rank]  (fp64 triangular solves, a warp per 4 columns)
+//   W  = L^-T (L^-1 C1),  L = F[piv, :rank]  (blocked fp64 triangular solves, 8 columns a block)
 // L L^T = h(K_S, K_S) because the pivot rows of the RPCholesky factor are the
 // Cholesky factor of the kernel matrix on the coreset (in pivot order).
 #include "wc_common.cuh"
@@ -33,8 +33,6 @@ __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict
         lrow[b] = (p >= 0 && b <= a) ? Fu[(int64_t)b * ldf + p] : 0.f;
 }
 
-constexpr int kCols = 4;  // right-hand-side columns per solving warp
-
 // C1 from the partial sums of the key splits, in fp64:
 //   C1[a, c] = e^M sum_s e^{m_s - M} O_s[a, c],  M = max_s m_s
 // written column-major, Ct[u, c, a], for the solves.  One block per (a, u).
@@ -60,113 +58,143 @@ __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t*
     }
 }
 
-// W = L^-T (L^-1 C1) for kCols right-hand sides of one unit, one warp, fp64,
-// in blocks of 32 rows.  Forward, block [a0, a0+32): lane i owns row a0+i,
-// subtracts L[a0+i, :a0] y[:a0] (its own row of L, independent loads), then the
-// 32 x 32 diagonal block is solved through shuffles.  Backward, blocks from the
-// last: lane i owns entry a0+i, subtracts sum_{b >= a0+32} L[b, a0+i] x_b (row
-// segments of L, coalesced across the warp), then the diagonal block.
-// y / x live in shared memory, [kCols][r].
-__global__ void __launch_bounds__(32) trsv_kernel(const float* __restrict__ Lg, const int32_t* __restrict__ rank,
-                                                  const double* __restrict__ Ct, float* W, int r, int dv) {
-    extern __shared__ double ys[];
+// W = L^-T (L^-1 C1) for NC right-hand-side columns of one unit, fp64, blocked
+// by 64 rows (right-looking).  The NC columns live in shared memory (Y, row
+// major [r][NC]) for the whole solve.
+//   forward, block K = [kb, kb + 64):  Y_K <- L_KK^-1 Y_K (one warp per column,
+//     lanes own rows kb + lane and kb + lane + 32, the diagonal block staged in
+//     shared memory), then every later row i: Y_i -= L[i, K] Y_K (one thread
+//     per row; a thread reads its row segment of L).
+//   backward, blocks from the last:  Y_K <- L_KK^-T Y_K, then every earlier row
+//     i: Y_i -= L[K, i]^T Y_K (threads over i read rows of L: coalesced).
+// Rows at and beyond the rank are left out; W rows there are written as zero.
+constexpr int kTB = 64;           // rows per diagonal block
+constexpr int kTrsmThreads = 256;
+
+template <int NC>
+__global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restrict__ Lg,
+                                                           const int32_t* __restrict__ rank,
+                                                           const double* __restrict__ Ct, float* W, int r, int dv) {
+    extern __shared__ double sm_d[];
+    double* Y = sm_d;                                        // [r][NC]
+    float* Ld = reinterpret_cast<float*>(Y + (size_t)r * NC);  // [kTB][kTB + 1] diagonal block
     const int u = blockIdx.y;
     const int wcols = dv + 1;
-    const int c0 = blockIdx.x * kCols;
-    const int nc = min(kCols, wcols - c0);
+    const int c0 = blockIdx.x * NC;
+    const int nc = min(NC, wcols - c0);
     const int k = rank[u];
     const float* L = Lg + (size_t)u * r * r;
     const double* C = Ct + (size_t)u * wcols * r;
     float* Wu = W + (size_t)u * r * wcols;
-    const int lane = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int e = tid; e < NC * k; e += kTrsmThreads) {
+        const int q = e / k, a = e - q * k;
+        Y[a * NC + q] = q < nc ? C[(size_t)(c0 + q) * r + a] : 0.0;
+    }
 
     // ---- forward: L y = c
-    for (int a0 = 0; a0 < k; a0 += 32) {
-        const int a = a0 + lane;
-        const bool live = a < k;
-        double acc[kCols];
+    for (int kb = 0; kb < k; kb += kTB) {
+        const int bs = min(kTB, k - kb);
+        __syncthreads();
+        for (int e = tid; e < kTB * kTB; e += kTrsmThreads) {
+            const int i = e / kTB, j = e % kTB;
+            Ld[i * (kTB + 1) + j] = (i < bs && j <= i) ? L[(size_t)(kb + i) * r + kb + j] : 0.f;
+        }
+        __syncthreads();
+        if (warp < NC) {
+            const int q = warp;
+            double y0 = lane < bs ? Y[(kb + lane) * NC + q] : 0.0;
+            double y1 = lane + 32 < bs ? Y[(kb + lane + 32) * NC + q] : 0.0;
+            for (int i = 0; i < bs; ++i) {
+                const double own = (i < 32) ? y0 : y1;
+                const double yi = __shfl_sync(0xffffffffu, own / (double)Ld[i * (kTB + 1) + i], i & 31);
+                if (lane == (i & 31)) {
+                    if (i < 32) y0 = yi;
+                    else y1 = yi;
+                }
+                if (lane > i) y0 -= (double)Ld[lane * (kTB + 1) + i] * yi;
+                if (lane + 32 > i) y1 -= (double)Ld[(lane + 32) * (kTB + 1) + i] * yi;
+            }
+            if (lane < bs) Y[(kb + lane) * NC + q] = y0;
+            if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
+        }
+        __syncthreads();
+        for (int i = kb + bs + tid; i < k; i += kTrsmThreads) {
+            double acc[NC];
 #pragma unroll
-        for (int q = 0; q < kCols; ++q) acc[q] = (live && q < nc) ? C[(size_t)(c0 + q) * r + a] : 0.0;
-        float lb[32];  // this row's entries in the diagonal block
-        if (live) {
-            const float* La = L + (size_t)a * r;
-#pragma unroll 8
-            for (int b = 0; b < a0; ++b) {
-                const double l = (double)La[b];
+            for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
+            const float* Li = L + (size_t)i * r + kb;
+            for (int b = 0; b < bs; ++b) {
+                const double l = (double)Li[b];
 #pragma unroll
-                for (int q = 0; q < kCols; ++q) acc[q] -= l * ys[q * r + b];
+                for (int q = 0; q < NC; ++q) acc[q] -= l * Y[(kb + b) * NC + q];
             }
 #pragma unroll
-            for (int t = 0; t < 32; ++t) lb[t] = (a0 + t < k) ? La[a0 + t] : 0.f;
-        } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t) lb[t] = 0.f;
+            for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
         }
-        const int rows = min(32, k - a0);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (i < rows) {
-                double yi[kCols];
-#pragma unroll
-                for (int q = 0; q < kCols; ++q) {
-                    const double v = (lane == i) ? acc[q] / (double)lb[i] : 0.0;
-                    yi[q] = __shfl_sync(0xffffffffu, v, i);
-                }
-                if (lane == i) {
-#pragma unroll
-                    for (int q = 0; q < kCols; ++q) ys[q * r + a] = yi[q];
-                }
-                if (lane > i) {
-                    const double l = (double)lb[i];
-#pragma unroll
-                    for (int q = 0; q < kCols; ++q) acc[q] -= l * yi[q];
-                }
-            }
-        }
-        __syncwarp();
     }
 
     // ---- backward: L^T x = y
-    for (int a0 = (k - 1) / 32 * 32; k > 0 && a0 >= 0; a0 -= 32) {
-        const int a = a0 + lane;
-        const bool live = a < k;
-        double acc[kCols];
-#pragma unroll
-        for (int q = 0; q < kCols; ++q) acc[q] = live ? ys[q * r + a] : 0.0;
-#pragma unroll 8
-        for (int b = a0 + 32; b < k; ++b) {
-            const double l = live ? (double)L[(size_t)b * r + a] : 0.0;
-#pragma unroll
-            for (int q = 0; q < kCols; ++q) acc[q] -= l * ys[q * r + b];
+    for (int kb = (k - 1) / kTB * kTB; k > 0 && kb >= 0; kb -= kTB) {
+        const int bs = min(kTB, k - kb);
+        __syncthreads();
+        for (int e = tid; e < kTB * kTB; e += kTrsmThreads) {
+            const int i = e / kTB, j = e % kTB;
+            Ld[i * (kTB + 1) + j] = (i < bs && j <= i) ? L[(size_t)(kb + i) * r + kb + j] : 0.f;
         }
-        float lt[32];  // lt[i] = L[a0 + i, a]: this entry's column of the diagonal block
-#pragma unroll
-        for (int i = 0; i < 32; ++i) lt[i] = (live && a0 + i < k) ? L[(size_t)(a0 + i) * r + a] : 0.f;
-        const int rows = min(32, k - a0);
-#pragma unroll
-        for (int i = 31; i >= 0; --i) {
-            if (i < rows) {
-                double xi[kCols];
-#pragma unroll
-                for (int q = 0; q < kCols; ++q) {
-                    const double v = (lane == i) ? acc[q] / (double)lt[i] : 0.0;
-                    xi[q] = __shfl_sync(0xffffffffu, v, i);
+        __syncthreads();
+        if (warp < NC) {
+            const int q = warp;
+            double y0 = lane < bs ? Y[(kb + lane) * NC + q] : 0.0;
+            double y1 = lane + 32 < bs ? Y[(kb + lane + 32) * NC + q] : 0.0;
+            for (int i = bs - 1; i >= 0; --i) {
+                const double own = (i < 32) ? y0 : y1;
+                const double xi = __shfl_sync(0xffffffffu, own / (double)Ld[i * (kTB + 1) + i], i & 31);
+                if (lane == (i & 31)) {
+                    if (i < 32) y0 = xi;
+                    else y1 = xi;
                 }
-                if (lane == i) {
-#pragma unroll
-                    for (int q = 0; q < kCols; ++q) ys[q * r + a] = xi[q];
-                }
-                if (lane < i) {
-                    const double l = (double)lt[i];
-#pragma unroll
-                    for (int q = 0; q < kCols; ++q) acc[q] -= l * xi[q];
-                }
+                if (lane < i) y0 -= (double)Ld[i * (kTB + 1) + lane] * xi;
+                if (lane + 32 < i) y1 -= (double)Ld[i * (kTB + 1) + lane + 32] * xi;
             }
+            if (lane < bs) Y[(kb + lane) * NC + q] = y0;
+            if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
         }
-        __syncwarp();
+        __syncthreads();
+        for (int i = tid; i < kb; i += kTrsmThreads) {
+            double acc[NC];
+#pragma unroll
+            for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
+            for (int b = 0; b < bs; ++b) {
+                const double l = (double)L[(size_t)(kb + b) * r + i];
+#pragma unroll
+                for (int q = 0; q < NC; ++q) acc[q] -= l * Y[(kb + b) * NC + q];
+            }
+#pragma unroll
+            for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
+        }
     }
-    for (int q = 0; q < nc; ++q)
-        for (int a = lane; a < r; a += 32) Wu[(size_t)a * wcols + c0 + q] = a < k ? (float)ys[q * r + a] : 0.f;
+    __syncthreads();
+    for (int e = tid; e < r * nc; e += kTrsmThreads) {
+        const int a = e / nc, q = e - a * nc;
+        Wu[(size_t)a * wcols + c0 + q] = a < k ? (float)Y[a * NC + q] : 0.f;
+    }
+}
+
+template <int NC>
+size_t trsm_smem(int r) {
+    return sizeof(double) * NC * (size_t)r + sizeof(float) * kTB * (kTB + 1);
+}
+
+template <int NC>
+wc_status launch_trsm_t(const Shape& s, const float* Lg, const int32_t* rank, const double* Ct, float* W,
+                        cudaStream_t st) {
+    const size_t smem = trsm_smem<NC>(s.r);
+    if (cudaFuncSetAttribute(trsm_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return WC_ERR_CUDA;
+    trsm_kernel<NC><<<dim3((s.dv + 1 + NC - 1) / NC, s.units), kTrsmThreads, smem, st>>>(Lg, rank, Ct, W, s.r, s.dv);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
 }  // namespace
@@ -211,12 +239,14 @@ wc_status launch_solve(const Shape& s, const int32_t* rank, float* W, char* ws, 
     merge_c1_kernel<<<dim3(s.r, s.units), 160, 0, st>>>(reinterpret_cast<const float*>(ws + L.c1part), rank, Ct,
                                                         s.nsplit, s.r, s.dv);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
-    const size_t smem = sizeof(double) * kCols * (size_t)s.r;
-    if (cudaFuncSetAttribute(trsv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return WC_ERR_CUDA;
-    trsv_kernel<<<dim3((s.dv + 1 + kCols - 1) / kCols, s.units), 32, smem, st>>>(
-        reinterpret_cast<const float*>(ws + L.lg), rank, Ct, W, s.r, s.dv);
-    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+    // as many right-hand sides per block as shared memory holds for this r
+    const float* Lg = reinterpret_cast<const float*>(ws + L.lg);
+    constexpr size_t kMax = 232448;
+    if (trsm_smem<8>(s.r) <= kMax) return launch_trsm_t<8>(s, Lg, rank, Ct, W, st);
+    if (trsm_smem<4>(s.r) <= kMax) return launch_trsm_t<4>(s, Lg, rank, Ct, W, st);
+    if (trsm_smem<2>(s.r) <= kMax) return launch_trsm_t<2>(s, Lg, rank, Ct, W, st);
+    if (trsm_smem<1>(s.r) <= kMax) return launch_trsm_t<1>(s, Lg, rank, Ct, W, st);
+    return WC_ERR_UNSUPPORTED;
 }
 
 }  // namespace wc
