@@ -36,10 +36,34 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->esize = s.dtype == WC_BF16 ? 2 : 4;
     o->nsplit = (s.n_k + kSplitKeys - 1) / kSplitKeys;
     o->r_pad = (s.r + 63) / 64 * 64;
+    if (s.bins < 0 || (s.center != 0 && s.center != 1)) return WC_ERR_INVALID;
+    o->bins = s.bins > 1 ? s.bins : 1;
+    if (s.n_k % o->bins || s.r % o->bins) return WC_ERR_INVALID;
+    o->center = s.center;
+    o->units_all = o->units;
+    o->n_all = s.n_k;
+    o->r_all = s.r;
     return WC_OK;
 }
 
+Shape bin_view(const Shape& s) {
+    Shape b = s;
+    if (s.bins <= 1) return b;
+    b.hkv = s.hkv * s.bins;
+    b.hq = s.hq * s.bins;
+    b.units = s.units_all * s.bins;
+    b.n = s.n_all / s.bins;
+    b.r = s.r_all / s.bins;
+    b.ldf = f_ld(b.n);
+    b.nsplit = (b.n + kSplitKeys - 1) / kSplitKeys;
+    b.r_pad = (b.r + 63) / 64 * 64;
+    return b;
+}
+
 WsLayout make_layout(const Shape& s) {
+    // Every region is sized from the caller's problem (units_all, n_all, r_all,
+    // bins) for the larger of its unit-view and bin-view needs, so the select,
+    // weights and attend launchers agree on the offsets whichever view they get.
     WsLayout L;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -47,25 +71,30 @@ WsLayout make_layout(const Shape& s) {
         off = align_up(off + bytes, kWsAlign);
         return at;
     };
-    const size_t U = (size_t)s.units;
+    const size_t U = (size_t)s.units_all, B = (size_t)s.bins;
+    const size_t n = (size_t)s.n_all, r = (size_t)s.r_all, nb = n / B, rb = r / B;
+    const size_t ldb = (size_t)f_ld((int32_t)nb);
+    const size_t nsb = (nb + kSplitKeys - 1) / kSplitKeys;
+    const size_t r_pad = (r + 63) / 64 * 64;
+    const size_t kt_unit = U * s.d * (size_t)f_ld((int32_t)n), kt_bin = U * B * s.d * ldb;
     L.status = take(256);
-    L.sync = take(sizeof(UnitSync) * U);
-    L.partials = take(sizeof(double) * U * 2 * kMaxBlocksPerUnit);
-    L.kt = take((size_t)s.esize * U * s.d * s.ldf);
-    L.lg = take(sizeof(float) * U * s.r * s.r);
-    L.c1part = take(sizeof(float) * U * s.nsplit * s.r * (s.dv + 2));
-    L.y = take(sizeof(double) * U * s.r * (s.dv + 1));
+    L.sync = take(sizeof(UnitSync) * U * B);
+    L.partials = take(sizeof(double) * U * B * 2 * kMaxBlocksPerUnit);
+    L.kt = take((size_t)s.esize * (kt_unit > kt_bin ? kt_unit : kt_bin));
+    L.lg = take(sizeof(float) * U * B * rb * rb);
+    L.c1part = take(sizeof(float) * U * B * nsb * rb * (s.dv + 2));
+    L.y = take(sizeof(double) * U * r * (s.dv + 1));
     const bool tc = s.dtype == WC_BF16;
-    L.v16 = take(tc ? 2 * U * s.n * s.dv : 0);
-    L.w16 = take(tc ? 2 * U * s.r * s.dv : 0);
+    L.v16 = take(tc ? 2 * U * n * s.dv : 0);
+    L.w16 = take(tc ? 2 * U * r * s.dv : 0);
     L.sigma = take(tc ? sizeof(float) * U * s.dv : 0);
-    L.wn = take(tc ? sizeof(float) * U * s.r_pad : 0);
+    L.wn = take(tc ? sizeof(float) * U * r_pad : 0);
     L.scratch_end = off;
-    L.piv = take(sizeof(int32_t) * U * s.r);
-    L.rank = take(sizeof(int32_t) * U);
-    L.f = take(sizeof(float) * U * s.r * s.ldf);
-    L.ks = take((size_t)s.esize * U * s.r * s.d);
-    L.w = take(sizeof(float) * U * s.r * (s.dv + 1));
+    L.piv = take(sizeof(int32_t) * U * r);
+    L.rank = take(sizeof(int32_t) * U * B);
+    L.f = take(sizeof(float) * U * B * rb * ldb);
+    L.ks = take((size_t)s.esize * U * r * s.d);
+    L.w = take(sizeof(float) * U * r * (s.dv + 1));
     L.forward_end = off;
     return L;
 }
@@ -106,7 +135,7 @@ wc_status wc_select(const wc_shape* shape, const void* K, int32_t* piv, float* F
     if (e != WC_OK) return e;
     if (!K || !piv || !F || !rank || !aligned16(K) || !aligned16(F) || !aligned16(piv)) return WC_ERR_INVALID;
     if ((e = check_ws(s, ws, ws_bytes, false)) != WC_OK) return e;
-    return launch_select(s, K, piv, F, rank, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+    return launch_select(bin_view(s), K, piv, F, rank, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
 }
 
 wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const int32_t* piv, const float* F,
@@ -119,9 +148,10 @@ wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const 
     if ((e = check_ws(s, ws, ws_bytes, false)) != WC_OK) return e;
     char* w = static_cast<char*>(ws);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((e = launch_gather(s, K, piv, F, rank, Ks, w, st)) != WC_OK) return e;
-    if ((e = launch_coreset_values(s, Ks, K, V, rank, w, st)) != WC_OK) return e;
-    return launch_solve(s, rank, W, w, st);
+    const Shape sb = bin_view(s);
+    if ((e = launch_gather(sb, K, piv, F, rank, Ks, w, st)) != WC_OK) return e;
+    if ((e = launch_coreset_values(sb, Ks, K, V, rank, w, st)) != WC_OK) return e;
+    return launch_solve(sb, rank, W, w, st);
 }
 
 wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const float* W, const int32_t* rank,

@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(kThreads) expmm_simt_kernel(const ExpmmArgs e)
         unit = (z / e.hq) * hkv + (z % e.hq) / e.group;
         a_valid = e.a_rows;
         b_lo = 0;
-        b_hi = e.rank[unit];
+        b_hi = e.all_keys ? e.b_rows : e.rank[unit];
     }
     const int a0 = blockIdx.x * BM;
     if (a0 >= a_valid) return;

@@ -70,6 +70,7 @@ struct TcArgs {
     int nsplit, split_len;
     int r, r_pad;
     int hq, group;
+    int all_keys;        // rownorm: all b_rows rows count (binned coresets), else rank[unit]
     float cb;            // beta * log2(e)
 };
 
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         unit = (z / args.hq) * hkv + (z % args.hq) / args.group;
         a_valid = args.a_rows;
         b_lo = 0;
-        b_hi = args.rank[unit];
+        b_hi = args.all_keys ? args.b_rows : args.rank[unit];
         a_row0 = z * args.a_head_rows + blockIdx.x * BM;
     }
     const int a0 = blockIdx.x * BM;
@@ -515,9 +516,9 @@ __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __
 // max_s |W[s, c]| and W16[s, c] = W[s, c] / sigma_c (fp16); wn[s] = W[s, dv]
 // padded with zeros to r_pad rows.  One block per unit.
 __global__ void weights_prep_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, __half* W16,
-                                    float* sigma, float* wn, int r, int r_pad, int dv) {
+                                    float* sigma, float* wn, int r, int r_pad, int dv, int all_keys) {
     const int u = blockIdx.x;
-    const int k = rank[u];
+    const int k = all_keys ? r : rank[u];
     const float* Wu = W + (size_t)u * r * (dv + 1);
     __shared__ float sg[256];
     for (int c = threadIdx.x; c < dv; c += blockDim.x) {
@@ -628,7 +629,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     __half* W16 = reinterpret_cast<__half*>(ws + Lw.w16);
     float* sigma = reinterpret_cast<float*>(ws + Lw.sigma);
     float* wn = reinterpret_cast<float*>(ws + Lw.wn);
-    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv);
+    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv, s.bins > 1);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
     CUtensorMap mA, mB, mC;
     if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
@@ -650,6 +651,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     a.r_pad = s.r_pad;
     a.hq = s.hq;
     a.group = s.hq / s.hkv;
+    a.all_keys = s.bins > 1;
     a.cb = (float)(s.beta * 1.4426950408889634);
     dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
     return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
@@ -660,7 +662,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
 // point that allocates nothing.
 wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
                               float* out, int* status, __half* W16, float* sigma, float* wn, cudaStream_t st) {
-    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv);
+    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv, s.bins > 1);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
     CUtensorMap mA, mB, mC;
     if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
@@ -682,6 +684,7 @@ wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, con
     a.r_pad = s.r_pad;
     a.hq = s.hq;
     a.group = s.hq / s.hkv;
+    a.all_keys = s.bins > 1;
     a.cb = (float)(s.beta * 1.4426950408889634);
     dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
     return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);

@@ -50,6 +50,8 @@ struct SelectArgs {
     double beta, eps;
     uint64_t seed;
     uint64_t timeout_ns;
+    int32_t bins;      // key bins per caller unit: unit u is bin u % bins of its unit
+    int32_t bin_keys;  // keys per bin (pivot indices are reported within the caller's unit)
 };
 
 // Shared-memory plan (bytes) for m rows, r pivots, d dims.
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
                 us->s = r0 + sl;
                 us->d_s = ds;
                 us->stop = stop;
-                if (!stop) a.piv[(size_t)unit * r + j] = r0 + sl;
+                if (!stop) a.piv[(size_t)unit * r + j] = r0 + sl + (unit % a.bins) * a.bin_keys;
                 __threadfence();
                 st_release_u32(&us->pivflag, (uint32_t)j + 1u);
                 bc.s = r0 + sl;
@@ -477,6 +479,8 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
 
     SelectArgs a;
     a.K = K; a.piv = piv; a.F = F; a.rank = rank;
+    a.bins = s.bins;
+    a.bin_keys = s.n;
     a.Kt = ws + L.kt;
     a.sync = reinterpret_cast<UnitSync*>(ws + L.sync);
     a.partials = reinterpret_cast<double*>(ws + L.partials);

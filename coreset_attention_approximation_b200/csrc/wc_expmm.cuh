@@ -17,6 +17,7 @@ struct ExpmmArgs {
     const void* C;  int64_t c_stride; int ldc;      // value rows (dtype, or fp32 W)
     const float* wcol;                              // rownorm: W[:, dv] with row stride ldc
     const int32_t* rank;                            // valid coreset rows per unit
+    int all_keys;                                   // rownorm: every one of the b_rows rows counts
     void* out;
     int d, dv, r;
     int nsplit, split_len;

@@ -56,9 +56,15 @@ struct Shape {
     int32_t esize;         // bytes per Q/K/V element
     int32_t nsplit;        // C1 partial sums
     int32_t r_pad;         // r rounded up to 64
+    int32_t bins;          // key bins per unit (1: none); select and weights run on the bin view
+    int32_t center;        // subtract each unit's mean key before the selection and the weights
+    // the caller's problem, the same in the unit view and the bin view (sizes the workspace)
+    int32_t units_all, n_all, r_all;
 };
 
 wc_status make_shape(const wc_shape* in, Shape* out);
+// The per-bin problem: units * bins units of n / bins keys and r / bins pivots.
+Shape bin_view(const Shape& s);
 WsLayout make_layout(const Shape& s);
 
 // Kernel launchers (each returns WC_OK or WC_ERR_CUDA / WC_ERR_UNSUPPORTED).

@@ -16,17 +16,22 @@ namespace wc {
 namespace {
 
 // Ks[u, a, :] = K[u, piv[a], :] and Lg[u, a, b] = F[u, b, piv[a]] (b <= a),
-// zero beyond rank.  One block per (a, u).
+// zero beyond rank.  One block per (a, u).  With bins, u is bin u % bins of its
+// caller unit: pivot indices count from the caller unit's first key, and Ks rows
+// beyond the bin's rank repeat the bin's first pivot key (their weights are
+// zero, and a real key's logit leaves the row maxima of the attention intact).
 template <typename T>
 __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict__ piv,
                               const float* __restrict__ F, const int32_t* __restrict__ rank, T* Ks,
-                              float* Lg, int n, int d, int r, int64_t ldf) {
+                              float* Lg, int n, int d, int r, int64_t ldf, int bins) {
     const int a = blockIdx.x, u = blockIdx.y;
     const int k = rank[u];
-    const int p = a < k ? piv[(size_t)u * r + a] : -1;
+    const int base = (u % bins) * n;  // the bin's first key within the caller's unit
+    const int p = a < k ? piv[(size_t)u * r + a] - base : -1;
+    const int pk = p >= 0 ? p : (bins > 1 && k > 0 ? piv[(size_t)u * r] - base : -1);
     T* ks = Ks + ((size_t)u * r + a) * d;
     for (int c = threadIdx.x; c < d; c += blockDim.x)
-        ks[c] = p >= 0 ? K[((size_t)u * n + p) * d + c] : T(0.f);
+        ks[c] = pk >= 0 ? K[((size_t)u * n + pk) * d + c] : T(0.f);
     float* lrow = Lg + ((size_t)u * r + a) * r;
     const float* Fu = F + (size_t)u * r * ldf;
     for (int b = threadIdx.x; b < r; b += blockDim.x)
@@ -207,10 +212,10 @@ wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const
     if (s.dtype == WC_BF16)
         gather_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(K), piv, F, rank,
                                                            static_cast<__nv_bfloat16*>(Ks), Lg, s.n, s.d, s.r,
-                                                           s.ldf);
+                                                           s.ldf, s.bins);
     else
         gather_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(K), piv, F, rank,
-                                                   static_cast<float*>(Ks), Lg, s.n, s.d, s.r, s.ldf);
+                                                   static_cast<float*>(Ks), Lg, s.n, s.d, s.r, s.ldf, s.bins);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 

@@ -35,7 +35,7 @@ class WcShape(ctypes.Structure):
         ("n_k", ctypes.c_int32), ("n_q", ctypes.c_int32), ("d", ctypes.c_int32),
         ("dv", ctypes.c_int32), ("r", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("scale", ctypes.c_float), ("eps_stop", ctypes.c_float), ("wait_timeout_ms", ctypes.c_uint32),
-        ("seed", ctypes.c_uint64),
+        ("seed", ctypes.c_uint64), ("bins", ctypes.c_int32), ("center", ctypes.c_int32),
     ]
 
 
@@ -90,9 +90,10 @@ def _stream(stream):
 
 
 def make_shape(batch, hq, hkv, n_k, n_q, d, dv, r, dtype, scale=0.0, eps_stop=0.0, seed=0,
-               wait_timeout_ms=0) -> WcShape:
+               wait_timeout_ms=0, bins=1, center=False) -> WcShape:
     code = {torch.float32: WC_F32, torch.bfloat16: WC_BF16}.get(dtype, dtype)
-    return WcShape(batch, hq, hkv, n_k, n_q, d, dv, r, code, scale, eps_stop, wait_timeout_ms, seed)
+    return WcShape(batch, hq, hkv, n_k, n_q, d, dv, r, code, scale, eps_stop, wait_timeout_ms, seed,
+                   int(bins), int(bool(center)))
 
 
 def shape_of(Q, K, V, r, **kw) -> WcShape:
@@ -127,10 +128,18 @@ def workspace(shape: WcShape, device, forward_room: bool = False) -> torch.Tenso
 
 def _outputs(shape: WcShape, device, dtype):
     B, Hkv, r, n = shape.batch, shape.hkv, shape.r, shape.n_k
+    nb = max(shape.bins, 1)
+    if nb > 1:
+        # bins: per-bin ranks and per-bin factors over each bin's keys
+        rank = torch.empty(B, Hkv, nb, dtype=torch.int32, device=device)
+        F = torch.empty(B, Hkv, nb, r // nb, f_ld(n // nb), dtype=torch.float32, device=device)
+    else:
+        rank = torch.empty(B, Hkv, dtype=torch.int32, device=device)
+        F = torch.empty(B, Hkv, r, f_ld(n), dtype=torch.float32, device=device)
     return dict(
         piv=torch.empty(B, Hkv, r, dtype=torch.int32, device=device),
-        rank=torch.empty(B, Hkv, dtype=torch.int32, device=device),
-        F=torch.empty(B, Hkv, r, f_ld(n), dtype=torch.float32, device=device),
+        rank=rank,
+        F=F,
         Ks=torch.empty(B, Hkv, r, shape.d, dtype=dtype, device=device),
         W=torch.empty(B, Hkv, r, shape.dv + 1, dtype=torch.float32, device=device),
     )

@@ -43,6 +43,29 @@
  *       out [B, Hq,  n_q, dv]   fp32
  *     Query head g reads kv head g / (Hq / Hkv) (grouped-query attention).
  *   - Results are deterministic for a given shape, seed and GPU.
+ *
+ * Bins (shape.bins = B > 1)
+ *   [same gist.science page, "Methodik" item 1, "Effizienz": the input is split
+ *    into B bins processed in parallel, selection time O(n r^2 / B^3 + n r d / B^2)]
+ *   Each unit's keys split into B contiguous bins of n_k / B keys; each bin
+ *   selects r / B pivots on its own keys and solves its own weights (Philox
+ *   unit index (b * Hkv + h) * B + bin), and attention runs over the union of
+ *   the bins' coresets.  Layouts change as follows:
+ *       piv [B, Hkv, r]         key indices within the unit; bin b's pivots at
+ *                               positions b r/B .. (b+1) r/B - 1, -1 beyond its rank
+ *       rank[B, Hkv, bins]      pivots accepted per bin
+ *       F   [B, Hkv, bins, r/B, wc_f_ld(n_k / B)]   each bin's factor over its keys
+ *       Ks, W                   as above (r rows per unit); rows of bin b beyond its
+ *                               rank hold a copy of the bin's first pivot key in Ks
+ *                               and zeros in W, so attention over all r rows equals
+ *                               attention over the accepted pivots
+ *
+ * Centring (shape.center = 1)
+ *   [same page, "Methodik" item 3: softmax attention is invariant to a global
+ *    centring of the keys, K <- K - mean(K)]
+ *   The selection and the weights use the centred keys of each unit; Ks holds
+ *   the keys as given (K[piv]), and attention with them equals attention with
+ *   the centred keys (the shift multiplies a query's row by one factor).
  */
 #ifndef WILDCAT_H
 #define WILDCAT_H
@@ -81,6 +104,11 @@ typedef struct {
                          is <= eps_stop * max_i H_ii; 0 selects 2^-20 */
     uint32_t wait_timeout_ms;  /* bound on every device-side wait; 0 selects 10000 */
     uint64_t seed;    /* Philox4x32-10 key of the pivot draws */
+    int32_t bins;     /* 0 or 1: one selection over each unit's n_k keys.  B > 1: the
+                         divide-and-conquer selection; see "Bins" above.  n_k and r
+                         must be multiples of B */
+    int32_t center;   /* 0: keys as given.  1: each unit's mean key is subtracted
+                         before the selection and the weights; see "Centring" above */
 } wc_shape;
 
 /* Row stride (elements) of F for n_k keys: n_k rounded up to a multiple of 8. */

@@ -213,13 +213,34 @@ def exact_attention(Q, K, V, beta: float) -> np.ndarray:
     return out
 
 
+def center_keys(K) -> np.ndarray:
+    """Centring of one unit's keys, K - mean(K) over the keys, in fp64.
+    [WildCat, gist.science summary, "Methodik" item 3: keys are re-centred by
+    subtracting their mean; softmax attention is invariant to it.]"""
+    K = _f64(K)
+    return K - K.mean(axis=0, keepdims=True)
+
+
 def forward(Q, K, V, r: int, seed: int = 0, beta: float | None = None,
-            eps_stop: float = DEFAULT_EPS_STOP, replay=None, units=None, threads: int | None = None):
+            eps_stop: float = DEFAULT_EPS_STOP, replay=None, units=None, threads: int | None = None,
+            bins: int = 1, center: bool = False):
     """Whole method over [B, Hq, nq, d] / [B, Hkv, n, d] / [B, Hkv, n, dv] inputs.
 
-    replay: optional (piv [B, Hkv, r], rank [B, Hkv]) decisions to replay
-    (see wc_oracle.h).  units: optional list of unit indices to compute (the
-    others are left as zeros / -1).  Returns a dict of numpy arrays.
+    replay: optional (piv [B, Hkv, r], rank [B, Hkv] (bins: [B, Hkv, bins]))
+    decisions to replay (see wc_oracle.h).  units: optional list of unit
+    indices to compute (the others are left as zeros / -1).
+
+    bins > 1 (the pages' divide-and-conquer selection, "Methodik" item 1,
+    "Effizienz"; the bin layout and per-bin weights are this build's reading):
+    each unit's keys split into `bins` contiguous bins of n / bins keys; bin b
+    runs RPCholesky with r / bins pivots on its keys (Philox unit index
+    u * bins + b) and Nystrom weights on its keys and values; attention runs over
+    the union of the bins' coresets.  F is then [B, Hkv, n, r] block diagonal
+    (bin b's keys x bin b's columns).
+
+    center: the selection and the weights use K - mean(K) per unit; attention
+    uses the centred coreset keys too (equal to the raw keys' result, by the
+    invariance).  Returns a dict of numpy arrays.
     """
     Qa, Ka, Va = _f64(Q), _f64(K), _f64(V)
     B, Hq, nq, d = Qa.shape
@@ -227,34 +248,49 @@ def forward(Q, K, V, r: int, seed: int = 0, beta: float | None = None,
     dv = Va.shape[-1]
     if beta is None:
         beta = default_beta(d)
+    nb = max(int(bins), 1)
+    if n % nb or r % nb:
+        raise ValueError("n and r must be multiples of bins")
+    nbk, rb = n // nb, r // nb
     group = Hq // Hkv
     nunits = B * Hkv
     piv = np.full((B, Hkv, r), -1, dtype=np.int32)
-    rank = np.zeros((B, Hkv), dtype=np.int32)
+    rank = np.zeros((B, Hkv, nb), dtype=np.int32)
     F = np.zeros((B, Hkv, n, r), dtype=np.float64)
     W = np.zeros((B, Hkv, r, dv + 1), dtype=np.float64)
     out = np.zeros((B, Hq, nq, dv), dtype=np.float64)
-    infos = [None] * nunits
+    infos = [None] * (nunits * nb)
     todo = list(range(nunits)) if units is None else list(units)
 
     def run(u):
         b, h = divmod(u, Hkv)
-        rp = rr = None
-        if replay is not None:
-            rp = np.asarray(replay[0])[b, h]
-            rr = int(np.asarray(replay[1])[b, h])
-        res = rpcholesky(Ka[b, h], r, beta, seed=seed, unit=u, eps_stop=eps_stop,
-                         replay_piv=rp, replay_rank=rr)
-        k = res["rank"]
-        piv[b, h] = res["piv"]
-        rank[b, h] = k
-        F[b, h] = res["F"]
-        infos[u] = res
-        if k > 0:
-            W[b, h, :k] = nystrom_weights(Ka[b, h], Va[b, h], res["piv"], k, beta)
-            Ks = Ka[b, h][res["piv"][:k]]
+        Ku = center_keys(Ka[b, h]) if center else Ka[b, h]
+        rows = []
+        for bb in range(nb):
+            ks, ke = bb * nbk, (bb + 1) * nbk
+            rp = rr = None
+            if replay is not None:
+                rp = np.asarray(replay[0])[b, h, bb * rb:(bb + 1) * rb].copy()
+                rp[rp >= 0] -= ks
+                rr_all = np.asarray(replay[1])
+                rr = int(rr_all[b, h, bb] if rr_all.ndim == 3 else rr_all[b, h])
+            res = rpcholesky(Ku[ks:ke], rb, beta, seed=seed, unit=u * nb + bb, eps_stop=eps_stop,
+                             replay_piv=rp, replay_rank=rr)
+            k = res["rank"]
+            pb = res["piv"].copy()
+            pb[pb >= 0] += ks
+            piv[b, h, bb * rb:(bb + 1) * rb] = pb
+            rank[b, h, bb] = k
+            F[b, h, ks:ke, bb * rb:(bb + 1) * rb] = res["F"]
+            infos[u * nb + bb] = res
+            if k > 0:
+                W[b, h, bb * rb:bb * rb + k] = nystrom_weights(Ku[ks:ke], Va[b, h, ks:ke], res["piv"], k, beta)
+                rows.extend(range(bb * rb, bb * rb + k))
+        if rows:
+            sel = piv[b, h, rows]
+            Ks = Ku[sel]
             for g in range(group):
-                out[b, h * group + g] = coreset_attend(Qa[b, h * group + g], Ks, W[b, h, :k], beta)
+                out[b, h * group + g] = coreset_attend(Qa[b, h * group + g], Ks, W[b, h, rows], beta)
         else:
             out[b, h * group:(h + 1) * group] = np.nan
 
@@ -265,4 +301,6 @@ def forward(Q, K, V, r: int, seed: int = 0, beta: float | None = None,
     else:
         with ThreadPoolExecutor(max_workers=nthreads) as ex:
             list(ex.map(run, todo))
+    if nb == 1:
+        rank = rank[..., 0]
     return dict(piv=piv, rank=rank, F=F, W=W, out=out, info=infos, beta=beta)

@@ -70,3 +70,47 @@ def compare(Q, K, V, r, seed=0, eps_stop=None, check_F=True, tol_w=None, **kw):
     if tol_w is not None:
         assert report["err_W"] <= tol_w, report
     return report
+
+
+def compare_next(Q, K, V, r, seed=0, bins=1, center=False, check_F=True, tol_w=None, **kw):
+    """compare() for the binned selection and key centring: per-bin pivots,
+    ranks and factors against the oracle's (replayed within the 1e-6 window),
+    W and the output within the dtype's tolerance."""
+    g = run_gpu(Q, K, V, r, seed=seed, bins=bins, center=center, **kw)
+    piv_g, rank_g = g["piv"].numpy(), g["rank"].numpy()
+    nb = max(bins, 1)
+    rank3 = rank_g.reshape(rank_g.shape[0], rank_g.shape[1], nb)
+    o = oracle.forward(Q, K, V, r, seed=seed, replay=(piv_g, rank3), bins=nb, center=center)
+    B, Hkv = rank3.shape[:2]
+    n = K.shape[2]
+    nbk, rb = n // nb, r // nb
+    orank = np.asarray(o["rank"]).reshape(B, Hkv, nb)
+    report = dict(replays=0, err_out=0.0, err_W=0.0, err_F=0.0)
+    for b in range(B):
+        for h in range(Hkv):
+            for bb in range(nb):
+                info = o["info"][(b * Hkv + h) * nb + bb]
+                assert info["failed_step"] == -1, (b, h, bb, info)
+                report["replays"] += info["n_replays"]
+                k = int(rank3[b, h, bb])
+                assert k == int(orank[b, h, bb]), (b, h, bb)
+                if check_F:
+                    Fg = g["F"][b, h].numpy().reshape(nb, rb, -1)[bb][:, :nbk].T if nb > 1 else \
+                        g["F"][b, h].numpy()[:, :n].T
+                    Fo = o["F"][b, h, bb * nbk:(bb + 1) * nbk, bb * rb:(bb + 1) * rb]
+                    report["err_F"] = max(report["err_F"], rel_err(Fg, Fo))
+                rows = slice(bb * rb, bb * rb + k)
+                if k > 0:
+                    report["err_W"] = max(report["err_W"], rel_err(g["W"][b, h].numpy()[rows], o["W"][b, h, rows]))
+                assert np.all(g["W"][b, h].numpy()[bb * rb + k:(bb + 1) * rb] == 0.0)
+            assert np.array_equal(piv_g[b, h], o["piv"][b, h])
+    tol = TOL_OUT[K.dtype]
+    for b in range(B):
+        for hq in range(Q.shape[1]):
+            report["err_out"] = max(report["err_out"], rel_err(g["out"][b, hq].numpy(), o["out"][b, hq]))
+    assert report["err_out"] <= tol, report
+    if check_F:
+        assert report["err_F"] <= 1e-5, report
+    if tol_w is not None:
+        assert report["err_W"] <= tol_w, report
+    return report
