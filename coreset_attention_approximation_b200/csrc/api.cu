@@ -40,6 +40,7 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->bins = s.bins > 1 ? s.bins : 1;
     if (s.n_k % o->bins || s.r % o->bins) return WC_ERR_INVALID;
     o->center = s.center;
+    if (o->center) return WC_ERR_UNSUPPORTED;  // the centring kernels are not built yet
     o->units_all = o->units;
     o->n_all = s.n_k;
     o->r_all = s.r;
