@@ -377,7 +377,7 @@ def kernel_breakdown(step):
         short = None
         m = re.search(r"expmm_(tc|simt)_kernel<[^>]*?(\d)>", name)
         if m:
-            short = ("weights_gemm", "attend_gemm")[int(m.group(2))]
+            short = "attend_gemm" if m.group(2) == "1" else "weights_gemm"  # modes 0, 2: weights; 1: attention
         else:
             for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
                              ("merge_c1", "merge_c1"), ("trsm_kernel", "solve"), ("weights_prep", "w_prep")):

@@ -13,7 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwildcat.so")
 OBJDIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "select.cu", "weights.cu", "expmm_simt.cu", "expmm_tc.cu", "attend.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "select.cu", "weights.cu", "expmm_simt.cu", "expmm_tc.cu", "attend.cu", "noalloc.cu",
+           "center.cu"]
 HEADERS = ["wc_common.cuh", "wc_internal.h", "wc_expmm.cuh", "wc_tc.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

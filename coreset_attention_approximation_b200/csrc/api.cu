@@ -40,7 +40,6 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->bins = s.bins > 1 ? s.bins : 1;
     if (s.n_k % o->bins || s.r % o->bins) return WC_ERR_INVALID;
     o->center = s.center;
-    if (o->center) return WC_ERR_UNSUPPORTED;  // the centring kernels are not built yet
     o->units_all = o->units;
     o->n_all = s.n_k;
     o->r_all = s.r;
@@ -81,7 +80,8 @@ WsLayout make_layout(const Shape& s) {
     L.status = take(256);
     L.sync = take(sizeof(UnitSync) * U * B);
     L.partials = take(sizeof(double) * U * B * 2 * kMaxBlocksPerUnit);
-    L.kt = take((size_t)s.esize * (kt_unit > kt_bin ? kt_unit : kt_bin));
+    // transposed keys for the selection: fp32 when centred (centred values are not bf16)
+    L.kt = take((size_t)(s.center ? 4 : s.esize) * (kt_unit > kt_bin ? kt_unit : kt_bin));
     L.lg = take(sizeof(float) * U * B * rb * rb);
     L.c1part = take(sizeof(float) * U * B * nsb * rb * (s.dv + 2));
     L.y = take(sizeof(double) * U * r * (s.dv + 1));
@@ -90,6 +90,12 @@ WsLayout make_layout(const Shape& s) {
     L.w16 = take(tc ? 2 * U * r * s.dv : 0);
     L.sigma = take(tc ? sizeof(float) * U * s.dv : 0);
     L.wn = take(tc ? sizeof(float) * U * r_pad : 0);
+    const size_t C = s.center ? 1 : 0;
+    L.kpart = take(C * sizeof(double) * U * ((n + kCenterChunk - 1) / kCenterChunk) * s.d);
+    L.kbar = take(C * sizeof(double) * U * s.d);
+    L.kk = take(C * sizeof(double) * U);
+    L.cdot = take(C * sizeof(double) * U * n);
+    L.bias = take(C * sizeof(float) * U * B * ((nb + 127) / 128 * 128));
     L.scratch_end = off;
     L.piv = take(sizeof(int32_t) * U * r);
     L.rank = take(sizeof(int32_t) * U * B);
@@ -136,7 +142,10 @@ wc_status wc_select(const wc_shape* shape, const void* K, int32_t* piv, float* F
     if (e != WC_OK) return e;
     if (!K || !piv || !F || !rank || !aligned16(K) || !aligned16(F) || !aligned16(piv)) return WC_ERR_INVALID;
     if ((e = check_ws(s, ws, ws_bytes, false)) != WC_OK) return e;
-    return launch_select(bin_view(s), K, piv, F, rank, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+    char* w = static_cast<char*>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (s.center && (e = launch_center(s, K, w, st)) != WC_OK) return e;
+    return launch_select(bin_view(s), K, piv, F, rank, w, st);
 }
 
 wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const int32_t* piv, const float* F,
@@ -150,9 +159,10 @@ wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const 
     char* w = static_cast<char*>(ws);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape sb = bin_view(s);
+    if (s.center && (e = launch_center(s, K, w, st)) != WC_OK) return e;
     if ((e = launch_gather(sb, K, piv, F, rank, Ks, w, st)) != WC_OK) return e;
     if ((e = launch_coreset_values(sb, Ks, K, V, rank, w, st)) != WC_OK) return e;
-    return launch_solve(sb, rank, W, w, st);
+    return launch_solve(sb, piv, rank, W, w, st);
 }
 
 wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const float* W, const int32_t* rank,

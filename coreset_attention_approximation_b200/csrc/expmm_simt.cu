@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kThreads) expmm_simt_kernel(const ExpmmArgs e)
     const T* B = static_cast<const T*>(e.B) + (size_t)unit * e.b_stride;
     const TC* C = static_cast<const TC*>(e.C) + (size_t)unit * e.c_stride;
     const float* wcol = e.wcol ? e.wcol + (size_t)unit * e.c_stride : nullptr;
+    const float* bias = e.bias ? e.bias + (size_t)unit * e.bias_stride : nullptr;
 
     const int tid = threadIdx.x, row = tid / 8, sub = tid % 8;
     for (int x = tid; x < BM * d; x += kThreads) {
@@ -79,7 +80,8 @@ __global__ void __launch_bounds__(kThreads) expmm_simt_kernel(const ExpmmArgs e)
             const int jj = sub + 8 * k;
             float acc = 0.f;
             for (int c = 0; c < d; ++c) acc = fmaf(As[row * lda + c], Bs[jj * lda + c], acc);
-            sk[k] = (b0 + jj < b_hi) ? acc * e.beta : -INFINITY;
+            const float bj = (bias && b0 + jj < b_hi) ? bias[b0 + jj] * 0.6931471805599453f : 0.f;
+            sk[k] = (b0 + jj < b_hi) ? fmaf(acc, e.beta, bj) : -INFINITY;
             mt = fmaxf(mt, sk[k]);
         }
 #pragma unroll

@@ -72,7 +72,14 @@ struct TcArgs {
     int hq, group;
     int all_keys;        // rownorm: all b_rows rows count (binned coresets), else rank[unit]
     float cb;            // beta * log2(e)
+    const float* bias;   // kModeBias: per-key logit bias (log2 units), [units][bias_stride]
+    int bias_stride;
 };
+
+// MODE: kExpmmPartial, kExpmmRownorm, or kModeBias = partial sums of
+// exp(beta <a, b_j> + bias_j) (the centred kernel: the bias tile arrives with
+// the value tile).
+constexpr int kModeBias = 2;
 
 template <int D, int DV>
 struct Smem {
@@ -121,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int z = blockIdx.z;
     int unit, a_valid, b_lo, b_hi, split = 0, a_row0;
-    if (MODE == kExpmmPartial) {
+    if (MODE != kExpmmRownorm) {
         unit = z;
         a_valid = args.rank[unit];
         split = blockIdx.y;
@@ -199,13 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     #pragma unroll
                         for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &fl[s], c * 64, brow);
                     } else {
-                        mbar_expect_tx(&fl[s], L::kC + (MODE == kExpmmRownorm ? BN * 4 : 0));
+                        mbar_expect_tx(&fl[s], L::kC + (MODE != kExpmmPartial ? BN * 4 : 0));
                         unsigned char* st = sm + L::C0 + s * L::kC;
     #pragma unroll
                         for (int c = 0; c < DV / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapC, &fl[s], c * 64, brow);
                         if (MODE == kExpmmRownorm)
                             bulk_load(sm + L::Wv + s * BN * 4, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN,
                                       BN * 4, &fl[s]);
+                        if (MODE == kModeBias)
+                            bulk_load(sm + L::Wv + s * BN * 4,
+                                      args.bias + (size_t)unit * args.bias_stride + b_lo + t * BN, BN * 4, &fl[s]);
                     }
                     issued = t + 1;
                 }
@@ -303,11 +313,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             // pass 1: the whole row of S into registers, and its maximum
             float sv[BN];
             float mt = -INFINITY;
+            if (ok && MODE == kModeBias) {
+                // the logit bias arrives with the value tile
+                ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
+                ok = __all_sync(0xffffffffu, ok);
+            }
             if (ok) {
                 tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < 4; ++h) tmem_ld32(tS + 32 * h, sv + 32 * h);
                 tmem_wait_ld();
+                if (MODE == kModeBias) {
+                    // logits in log2 units, biased: S cb + bias_j (pass 2 then only subtracts the reference)
+                    const float* bv = reinterpret_cast<const float*>(sm + L::Wv + (t % NC) * BN * 4);
+#pragma unroll
+                    for (int j = 0; j < BN; j += 4) {
+                        const float4 f = lds_f4_ordered(bv + j);
+                        sv[j] = fmaf(sv[j], cb, f.x);
+                        sv[j + 1] = fmaf(sv[j + 1], cb, f.y);
+                        sv[j + 2] = fmaf(sv[j + 2], cb, f.z);
+                        sv[j + 3] = fmaf(sv[j + 3], cb, f.w);
+                    }
+                }
                 if (valid < BN) {
 #pragma unroll
                     for (int j = 0; j < BN; ++j)
@@ -319,7 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 8; j < BN; ++j) mq[j & 7] = fmaxf(mq[j & 7], sv[j]);
                 mt = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
-                           fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7]))) * cb;
+                           fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
+                if (MODE != kModeBias) mt *= cb;
             }
             // the reference after tile t - 1 (decided by the partner)
             if (t > 0) {
@@ -372,7 +400,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        const float p0 = ex2_ordered(fmaf(sh[j], cb, nm)), p1 = ex2_ordered(fmaf(sh[j + 1], cb, nm));
+                        float p0, p1;
+                        if (MODE == kModeBias) {
+                            p0 = ex2_ordered(sh[j] + nm);
+                            p1 = ex2_ordered(sh[j + 1] + nm);
+                        } else {
+                            p0 = ex2_ordered(fmaf(sh[j], cb, nm));
+                            p1 = ex2_ordered(fmaf(sh[j + 1], cb, nm));
+                        }
                         if (MODE == kExpmmRownorm)
                             lp[(j >> 1) & 3] = fmaf(p1, w[j + 1], fmaf(p0, w[j], lp[(j >> 1) & 3]));
                         else
@@ -444,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // has completed): each warp stages half of the columns of its 32 rows,
         // then the 256 softmax threads copy the block's rows, which are
         // contiguous in global memory, with coalesced stores.
-        constexpr int SST = (MODE == kExpmmPartial) ? DV + 2 : DV + 4;   // staged row stride (floats)
+        constexpr int SST = (MODE != kExpmmRownorm) ? DV + 2 : DV + 4;   // staged row stride (floats)
         float* stg = reinterpret_cast<float*>(sm + L::C0);
         const bool have_o = ok && T > 0;
         const uint32_t tO = tO0 + lanes + par * (DV / 2);
@@ -462,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0.f;
             }
-            if (MODE == kExpmmPartial) {
+            if (MODE != kExpmmRownorm) {
                 // staged rows are DV + 2 floats apart (the global layout): 8-byte aligned
 #pragma unroll
                 for (int c = 0; c < 32; c += 2)
@@ -477,12 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        if (MODE == kExpmmPartial && last) *reinterpret_cast<float2*>(stg + row * SST + DV) = make_float2(lt, mO * kLn2);
+        if (MODE != kExpmmRownorm && last) *reinterpret_cast<float2*>(stg + row * SST + DV) = make_float2(lt, mO * kLn2);
         softmax_sync();                         // all 8 softmax warps have staged their part
         const int rows = min(BM, a_valid - a0);
         const int st = tid - 4 * 32;            // 0 .. 255
         if (ok) {
-            if (MODE == kExpmmPartial) {
+            if (MODE != kExpmmRownorm) {
                 // rows a0 .. of this split are one contiguous run of rows * (DV + 2) floats
                 float2* dst = reinterpret_cast<float2*>(static_cast<float*>(args.out) +
                                                         (((size_t)unit * args.nsplit + split) * args.r + a0) * (DV + 2));
@@ -620,6 +655,11 @@ wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K
     a.group = 1;
     a.cb = (float)(s.beta * 1.4426950408889634);
     dim3 grid((s.r + TILES * BM - 1) / (TILES * BM), s.nsplit, s.units);
+    if (s.center) {
+        a.bias = reinterpret_cast<const float*>(ws + Lw.bias);
+        a.bias_stride = center_bias_stride(s);
+        return launch_tc<kModeBias>(s.d, s.dv, mA, mB, mC, a, grid, st);
+    }
     return launch_tc<kExpmmPartial>(s.d, s.dv, mA, mB, mC, a, grid, st);
 }
 

@@ -24,6 +24,8 @@
 // Blocks of one unit wait on each other, so a wave with C > 1 is launched
 // cooperatively (all blocks co-resident); every wait gives up after the
 // shape's timeout and records WC_ERR_TIMEOUT.
+#include <type_traits>
+
 #include "wc_common.cuh"
 #include "wc_internal.h"
 
@@ -52,6 +54,7 @@ struct SelectArgs {
     uint64_t timeout_ns;
     int32_t bins;      // key bins per caller unit: unit u is bin u % bins of its unit
     int32_t bin_keys;  // keys per bin (pivot indices are reported within the caller's unit)
+    const double* kbar;  // centring: mean key of each caller unit ([units / bins][d]), else null
 };
 
 // Shared-memory plan (bytes) for m rows, r pivots, d dims.
@@ -199,7 +202,9 @@ __device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, 
     }
 }
 
-template <typename T>
+// T: element type of K; TK: of the transposed copy that every step streams
+// (T, or fp32 when the keys are centred).
+template <typename T, typename TK>
 __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x;
@@ -220,13 +225,15 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     __shared__ Bcast bc;
 
     const T* K = static_cast<const T*>(a.K) + (size_t)unit * n * d;
-    T* Kt = static_cast<T*>(a.Kt) + (size_t)unit * d * ldf;
+    TK* Kt = static_cast<TK*>(a.Kt) + (size_t)unit * d * ldf;
+    const double* kb = a.kbar ? a.kbar + (size_t)(unit / a.bins) * d : nullptr;
     float* F = a.F + (size_t)unit * r * ldf;
     UnitSync* us = a.sync + unit;
     double* part = a.partials + (size_t)unit * 2 * kMaxBlocksPerUnit;
     int* status = a.status;
 
     // ---- initial residual: d_i = H_ii = exp(beta |k_i|^2); transpose the slice
+    // (centred: k_i - kbar, in fp64 for the diagonal, stored as fp32)
     double lmax = 0.0;
     for (int il = tid; il < ng * kGroup; il += kThreads) {
         const int i = r0 + il;
@@ -235,14 +242,16 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             double ss = 0.0;
             for (int c = 0; c < d; ++c) {
                 const T v = krow[c];
-                const double x = (double)to_f32(v);
+                double x = (double)to_f32(v);
+                if (kb) x -= kb[c];
                 ss += x * x;
-                Kt[(int64_t)c * ldf + i] = v;
+                if constexpr (std::is_same<T, TK>::value) Kt[(int64_t)c * ldf + i] = kb ? TK((float)x) : v;
+                else Kt[(int64_t)c * ldf + i] = (TK)(float)x;
             }
             dg[il] = exp(a.beta * ss);
             lmax = fmax(lmax, dg[il]);
         } else {
-            for (int c = 0; c < d; ++c) Kt[(int64_t)c * ldf + i] = T(0.f);
+            for (int c = 0; c < d; ++c) Kt[(int64_t)c * ldf + i] = TK(0.f);
             dg[il] = 0.0;
         }
         ispiv[il] = 0;
@@ -358,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         const double ds = bc.d_s;
 
         // 3. pivot key and F[s, 0..j) into shared memory
-        for (int c = tid; c < d; c += kThreads) ks[c] = (double)to_f32(K[(size_t)s * d + c]);
+        for (int c = tid; c < d; c += kThreads) ks[c] = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
         for (int c = tid; c < j; c += kThreads) fs[c] = ld_cg_f32(F + (int64_t)c * ldf + s);
         __syncthreads();
 
@@ -369,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             const int il0 = g * kGroup;
             const int i0 = r0 + il0;
             double dot[8], cor[8];
-            key_dots<T>(Kt + i0, ldf, d, ks, dot);
+            key_dots<TK>(Kt + i0, ldf, d, ks, dot);
             correction(F + i0, ldf, j, fs, cor);
             float out[8];
 #pragma unroll
@@ -424,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     }
 }
 
-template <typename T>
+template <typename T, typename TK>
 wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank, char* ws,
                           cudaStream_t st) {
     const WsLayout L = make_layout(s);
@@ -440,7 +449,7 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     int m_max = (int)(((size_t)max_smem - fixed) / 9) / kGroup * kGroup;
     m_max = m_max > (1 << 20) ? (1 << 20) : m_max;
 
-    auto kern = rpcholesky_kernel<T>;
+    auto kern = rpcholesky_kernel<T, TK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem - 1024) != cudaSuccess)
         return WC_ERR_CUDA;
     auto blocks_per_sm = [&](int m) {
@@ -481,6 +490,7 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     a.K = K; a.piv = piv; a.F = F; a.rank = rank;
     a.bins = s.bins;
     a.bin_keys = s.n;
+    a.kbar = s.center ? reinterpret_cast<const double*>(ws + L.kbar) : nullptr;
     a.Kt = ws + L.kt;
     a.sync = reinterpret_cast<UnitSync*>(ws + L.sync);
     a.partials = reinterpret_cast<double*>(ws + L.partials);
@@ -522,8 +532,11 @@ __global__ void wait_selftest_kernel(UnitSync* sync, int* status, uint64_t timeo
 
 wc_status launch_select(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank, char* ws,
                         cudaStream_t st) {
-    if (s.dtype == WC_BF16) return launch_select_t<__nv_bfloat16>(s, K, piv, F, rank, ws, st);
-    return launch_select_t<float>(s, K, piv, F, rank, ws, st);
+    if (s.dtype == WC_BF16) {
+        if (s.center) return launch_select_t<__nv_bfloat16, float>(s, K, piv, F, rank, ws, st);
+        return launch_select_t<__nv_bfloat16, __nv_bfloat16>(s, K, piv, F, rank, ws, st);
+    }
+    return launch_select_t<float, float>(s, K, piv, F, rank, ws, st);
 }
 
 wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st) {

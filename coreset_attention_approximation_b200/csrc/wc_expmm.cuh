@@ -18,6 +18,8 @@ struct ExpmmArgs {
     const float* wcol;                              // rownorm: W[:, dv] with row stride ldc
     const int32_t* rank;                            // valid coreset rows per unit
     int all_keys;                                   // rownorm: every one of the b_rows rows counts
+    const float* bias;                              // partial: per-key logit bias (log2 units) or null
+    int bias_stride;                                // floats per unit of bias
     void* out;
     int d, dv, r;
     int nsplit, split_len;

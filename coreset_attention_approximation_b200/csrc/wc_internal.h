@@ -12,6 +12,7 @@ namespace wc {
 
 constexpr int kMaxBlocksPerUnit = 512;   // select: thread blocks that share one unit
 constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1
+constexpr int kCenterChunk = 1024;       // centring: keys per partial column sum
 constexpr int kWsAlign = 256;
 
 // One per unit, in the workspace; zeroed before every select launch.
@@ -39,6 +40,12 @@ struct WsLayout {
     size_t w16;       // half[units][r][dv]     column-scaled weights for attention
     size_t sigma;     // float[units][dv]       their column scales
     size_t wn;        // float[units][r_pad]    normaliser column W[:, dv]
+    // centring (sizes 0 unless shape.center): per caller unit
+    size_t kpart;     // double[units][n / kCenterChunk][d]  partial column sums
+    size_t kbar;      // double[units][d]       mean key
+    size_t kk;        // double[units]          |mean|^2
+    size_t cdot;      // double[units][n]       <k_i, mean>
+    size_t bias;      // float[units * bins][stride]  -beta log2(e) <k_i, mean> per bin, padded
     size_t scratch_end;
     // room for outputs that wc_forward keeps in the workspace when not given
     size_t piv, rank, f, ks, w;
@@ -74,7 +81,12 @@ wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const
                         const int32_t* rank, void* Ks, char* ws, cudaStream_t st);
 wc_status launch_coreset_values(const Shape& s, const void* Ks, const void* K, const void* V,
                                 const int32_t* rank, char* ws, cudaStream_t st);
-wc_status launch_solve(const Shape& s, const int32_t* rank, float* W, char* ws, cudaStream_t st);
+wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, float* W, char* ws,
+                       cudaStream_t st);
+// Centring statistics of every caller unit (mean key, |mean|^2, <k_i, mean>,
+// the per-bin logit bias); `s` may be either view.
+wc_status launch_center(const Shape& s, const void* K, char* ws, cudaStream_t st);
+int center_bias_stride(const Shape& s);  // floats per bin row of the bias
 wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const float* W,
                         const int32_t* rank, float* out, char* ws, cudaStream_t st);
 wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st);

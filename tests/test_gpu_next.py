@@ -73,3 +73,44 @@ def test_bins_invalid_shapes_are_refused():
         wildcat.forward(Q, K, V, w.r, bins=3)          # n = 1024 is not a multiple of 3
     with pytest.raises(wildcat.WildcatError):
         wildcat.forward(Q, K, V, 66, bins=4)           # r = 66 is not a multiple of 4
+
+
+def _offset(w, seed, shift):
+    """The workload's inputs with one common vector added to every key (the
+    case centring exists for: the kernel matrix changes, attention does not)."""
+    Q, K, V = make_inputs(w, seed=seed)
+    g = torch.Generator().manual_seed(seed + 100)
+    c = torch.randn(K.shape[-1], generator=g, dtype=torch.float64) * shift
+    return Q, (K.double() + c).to(K.dtype), V
+
+
+def test_center_tiny_fp32():
+    w = WORKLOADS["tiny"]
+    compare_next(*_offset(w, 0, 0.5), w.r, seed=0, center=True, tol_w=1e-5)
+
+
+def test_center_vit():
+    w = WORKLOADS["vit"].replace(batch=4)
+    compare_next(*_offset(w, 1, 0.3), w.r, seed=1, center=True, tol_w=2e-3)
+
+
+def test_center_diffusion_mixture():
+    w = WORKLOADS["diffusion"].replace(batch=1, hq=4, hkv=4)
+    compare_next(*make_inputs(w), w.r, seed=2, center=True, tol_w=2e-3)
+
+
+def test_center_with_bins_kv():
+    w = WORKLOADS["kv"].replace(hq=8, hkv=2, n_k=8192, r=256)
+    compare_next(*_offset(w, 3, 0.2), w.r, seed=3, bins=4, center=True, tol_w=2e-3)
+
+
+def test_center_changes_the_selection_but_not_exactness():
+    # A large common key offset: without centring the kernel matrix is dominated
+    # by the offset; with it the run matches the oracle on the centred keys and
+    # the output still approximates the same attention.
+    w = WORKLOADS["vit"].replace(batch=1, hq=2, hkv=2, n_k=512, n_q=64, r=64)
+    Q, K, V = _offset(w, 4, 1.0)
+    a = run_gpu(Q, K, V, w.r, seed=4, center=True)
+    b = run_gpu(Q, K, V, w.r, seed=4)
+    assert not torch.equal(a["piv"], b["piv"])
+    compare_next(Q, K, V, w.r, seed=4, center=True, tol_w=2e-3)
