@@ -52,20 +52,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def select_bytes(w) -> float:
-    """Algorithmic bytes of one select launch: per unit and pivot step j, one
-    read of K (n d s_K), of the factor prefix F[:, :j] (4 n j) and one write of
-    the new column (4 n)."""
-    sk = 2 if w.dtype == "bf16" else 4
-    n, r, d = w.n_k, w.r, w.d
+def select_bytes(w, bins: int = 1, center: bool = False) -> float:
+    """Algorithmic bytes of one select launch: per unit (per bin with bins) and
+    pivot step j, one read of K (n d s_K), of the factor prefix F[:, :j] (4 n j)
+    and one write of the new column (4 n).  Centred keys stream as fp32."""
+    sk = 2 if (w.dtype == "bf16" and not center) else 4
+    n, r, d = w.n_k // bins, w.r // bins, w.d
     per_unit = n * r * d * sk + 2.0 * n * r * (r - 1) + 4.0 * n * r
-    return per_unit * w.batch * w.hkv
+    return per_unit * w.batch * w.hkv * bins
 
 
-def gemm_flops(w) -> tuple[float, float]:
-    """Tensor-core contraction flops: C1 = exp(K_S K^T)[V|1] per unit and
-    A = exp(Q K_S^T) W per query head, the [V|1] column counted."""
-    f1 = 2.0 * w.r * w.n_k * (w.d + w.dv + 1) * w.batch * w.hkv
+def gemm_flops(w, bins: int = 1) -> tuple[float, float]:
+    """Tensor-core contraction flops: C1 = exp(K_S K^T)[V|1] per unit (per bin:
+    r/B coreset rows against n/B keys) and A = exp(Q K_S^T) W per query head
+    over all r coreset rows, the [V|1] column counted."""
+    f1 = 2.0 * w.r * w.n_k * (w.d + w.dv + 1) * w.batch * w.hkv / bins
     f2 = 2.0 * w.n_q * w.r * (w.d + w.dv + 1) * w.batch * w.hq
     return f1, f2
 
@@ -166,21 +167,27 @@ def shard_seed(seed: int, rank: int) -> int:
 
 # ------------------------------------------------------------------ oracle sample
 
-def oracle_sample(w, r_s: int = 512, nq_s: int = 4096):
+def oracle_sample(w, r_s: int = 512, nq_s: int = 4096, bins: int = 1, center: bool = False):
     """Time the CPU oracle on a bounded sample of workload `w` and scale it to
     the whole workload.  Sample: unit 0, select steps 0..r_s-1 (the select's
     cost is n * sum_j (d + j) multiply-adds, so its time scales by that count),
     the weights on those r_s pivots (C1 dominates: linear in r) and attention
-    for nq_s queries of one head (linear in queries and in r)."""
+    for nq_s queries of one head (linear in queries and in r).  With bins the
+    select and weights sample is bin 0 of unit 0 (n/B keys, r/B pivots), scaled
+    by units x B; attention still covers r coreset rows."""
     import numpy as np
 
     import oracle
 
     Q, K, V = make_inputs(w.replace(batch=1, hq=w.hq // w.hkv, hkv=1))
     beta = 1.0 / math.sqrt(w.d)
-    r_s = min(r_s, w.r)
+    nb, rb = w.n_k // bins, w.r // bins
+    r_s = min(r_s, rb)
     nq_s = min(nq_s, w.n_q)
     Kn, Vn = K[0, 0].double().numpy(), V[0, 0].double().numpy()
+    if center:
+        Kn = oracle.center_keys(Kn)
+    Kn, Vn = Kn[:nb], Vn[:nb]
     t0 = time.perf_counter()
     sel = oracle.rpcholesky(Kn, r_s, beta, seed=0, unit=0)
     t1 = time.perf_counter()
@@ -191,12 +198,12 @@ def oracle_sample(w, r_s: int = 512, nq_s: int = 4096):
     t3 = time.perf_counter()
 
     def sel_work(r):
-        return w.n_k * (r * w.d + r * (r - 1) / 2.0)
+        return nb * (r * w.d + r * (r - 1) / 2.0)
 
-    units = w.batch * w.hkv
+    units = w.batch * w.hkv * bins
     heads = w.batch * w.hq
-    t_sel = (t1 - t0) * sel_work(w.r) / sel_work(r_s)
-    t_w = (t2 - t1) * w.r / r_s
+    t_sel = (t1 - t0) * sel_work(rb) / sel_work(r_s)
+    t_w = (t2 - t1) * rb / r_s
     t_att = (t3 - t2) * (w.n_q / nq_s) * (w.r / r_s)
     total = units * (t_sel + t_w) + heads * t_att
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
@@ -205,7 +212,8 @@ def oracle_sample(w, r_s: int = 512, nq_s: int = 4096):
         "unit": "tokens/s",
         "cores": cores,
         "kind": "oracle",
-        "sample": (f"{w.name}: unit 0 of {units}; select steps 0..{r_s - 1} of {w.r} "
+        "sample": (f"{w.name}{f' bins={bins}' if bins > 1 else ''}{' centred' if center else ''}: "
+                   f"unit 0 of {units}; select steps 0..{r_s - 1} of {rb} "
                    f"({t1 - t0:.1f} s, scaled by n*sum_j(d+j)); weights on {r_s} pivots ({t2 - t1:.1f} s, "
                    f"scaled x r/{r_s}); attend {nq_s} queries ({t3 - t2:.1f} s, scaled x n_q/{nq_s} x r/{r_s}); "
                    f"whole-workload estimate {total:.0f} s"),
@@ -223,7 +231,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     Qh, Kh, Vh = make_inputs(w, seed=shard_seed(args.seed, rank))
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
-    shape = wildcat.shape_of(Q, K, V, w.r, seed=args.seed)
+    shape = wildcat.shape_of(Q, K, V, w.r, seed=args.seed, bins=args.bins, center=args.center)
     ws = wildcat.workspace(shape, dev)
     o = wildcat._outputs(shape, dev, K.dtype)
     out = torch.empty(w.batch, w.hq, w.n_q, w.dv, dtype=torch.float32, device=dev)
@@ -290,7 +298,7 @@ def run_ours(args, world, rank, local):
         Q.copy_(Qp, non_blocking=True)
         K.copy_(Kp, non_blocking=True)
         V.copy_(Vp, non_blocking=True)
-        wildcat.forward(Q, K, V, w.r, seed=args.seed, ws=ws, outputs=outputs)
+        wildcat.forward(Q, K, V, w.r, seed=args.seed, ws=ws, outputs=outputs, bins=args.bins, center=args.center)
         outp.copy_(out, non_blocking=True)
 
     e2e_step()
@@ -311,11 +319,12 @@ def run_ours(args, world, rank, local):
 
     peaks, which = load_peaks()
     sel_avg = sum(sel_ms) / len(sel_ms)
-    sb = select_bytes(w)
+    sb = select_bytes(w, args.bins, args.center)
     achieved = sb / (sel_avg * 1e-3) / 1e9
-    f1, f2 = gemm_flops(w)
+    f1, f2 = gemm_flops(w, args.bins)
     wts_avg, att_avg = sum(wts_ms) / len(wts_ms), sum(att_ms) / len(att_ms)
-    traffic = SELECT_DRAM_BYTES_PER_UNIT[w.name] * w.batch * w.hkv if w.name in SELECT_DRAM_BYTES_PER_UNIT else None
+    captured = w.name in SELECT_DRAM_BYTES_PER_UNIT and args.bins == 1 and not args.center
+    traffic = SELECT_DRAM_BYTES_PER_UNIT[w.name] * w.batch * w.hkv if captured else None
     tokens = w.batch * w.n_q * world
     res = {
         "metric": METRIC,
@@ -333,6 +342,7 @@ def run_ours(args, world, rank, local):
         "config": {
             "workload": w.name, "batch": w.batch, "heads_q": w.hq, "heads_kv": w.hkv, "n_k": w.n_k,
             "n_q": w.n_q, "d": w.d, "dv": w.dv, "r": w.r, "keys": w.keys, "seed": args.seed,
+            "bins": args.bins, "center": bool(args.center),
             "l2": "inputs and factor larger than L2 (no flush)",
             "parallelism": f"independent units per rank x{world}",
         },
@@ -347,7 +357,7 @@ def run_ours(args, world, rank, local):
         "kernels_ms": kernels,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (CENTER_LAUNCHES if args.center else 0)) * args.steps,
         "clocks": clocks.summary(),
     }
     return res
@@ -356,6 +366,8 @@ def run_ours(args, world, rank, local):
 # select (1 cooperative wave here), gather, fp16 copy of V, C1 exp-GEMM, merge of
 # the C1 partials, triangular solves, weight preparation, attention exp-GEMM
 LAUNCHES_PER_STEP = 8
+# centring: column sums, mean, key-mean dots, once in the select and once in the weights
+CENTER_LAUNCHES = 6
 
 
 def kernel_breakdown(step):
@@ -404,11 +416,11 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     for _ in range(args.warmup):
-        oracle_sample(w, r_s=64, nq_s=256)
+        oracle_sample(w, r_s=64, nq_s=256, bins=args.bins, center=args.center)
     vals = []
     last = None
     for _ in range(args.steps):
-        last = oracle_sample(w, r_s=args.ref_pivots, nq_s=4096)
+        last = oracle_sample(w, r_s=args.ref_pivots, nq_s=4096, bins=args.bins, center=args.center)
         vals.append(last["value"])
     v = statistics.median(vals)
     return {
@@ -416,7 +428,8 @@ def run_reference(args, world, rank):
         "warmup": args.warmup, "ms_per_step": w.batch * w.n_q / v * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator; no dataset)",
         "config": {"workload": w.name, "batch": w.batch, "heads_q": w.hq, "heads_kv": w.hkv, "n_k": w.n_k,
-                   "n_q": w.n_q, "d": w.d, "dv": w.dv, "r": w.r, "keys": w.keys, "seed": args.seed},
+                   "n_q": w.n_q, "d": w.d, "dv": w.dv, "r": w.r, "keys": w.keys, "seed": args.seed,
+                   "bins": args.bins, "center": bool(args.center)},
         "impl": "reference",
         "cpu_baseline": {k: last[k] for k in ("value", "unit", "cores", "kind", "sample")} | {"value": v},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -433,6 +446,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-pivots", type=int, default=512, help="select steps in the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bins", type=int, default=1,
+                    help="divide-and-conquer selection: B key bins per head (n and r multiples of B)")
+    ap.add_argument("--center", action="store_true", help="centre the keys before selection and weights")
     args = ap.parse_args()
     if args.warmup < 3:
         print("note: warm-up raised to 3 steps", file=sys.stderr)
@@ -445,7 +461,8 @@ def main():
         else:
             res = run_ours(args, world, rank, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
-                cb = oracle_sample(WORKLOADS[args.workload], r_s=args.ref_pivots)
+                cb = oracle_sample(WORKLOADS[args.workload], r_s=args.ref_pivots, bins=args.bins,
+                                   center=args.center)
                 res["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
