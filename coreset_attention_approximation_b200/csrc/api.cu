@@ -83,7 +83,7 @@ WsLayout make_layout(const Shape& s) {
     // transposed keys for the selection: fp32 when centred (centred values are not bf16)
     L.kt = take((size_t)(s.center ? 4 : s.esize) * (kt_unit > kt_bin ? kt_unit : kt_bin));
     L.lg = take(sizeof(float) * U * B * rb * rb);
-    L.c1part = take(sizeof(float) * U * B * nsb * rb * (s.dv + 2));
+    L.c1part = take(sizeof(float) * U * B * nsb * rb * c1_row(s.dv));
     L.y = take(sizeof(double) * U * r * (s.dv + 1));
     const bool tc = s.dtype == WC_BF16;
     L.v16 = take(tc ? 2 * U * n * s.dv : 0);

@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) expmm_simt_kernel(const ExpmmArgs e)
     const int a = a0 + row;
     if (a >= a_valid) return;
     if (MODE == kExpmmPartial) {
-        float* out = static_cast<float*>(e.out) + (((size_t)unit * e.nsplit + split) * e.r + a) * (dv + 2);
+        float* out = static_cast<float*>(e.out) + (((size_t)unit * e.nsplit + split) * e.r + a) * c1_row(dv);
 #pragma unroll
         for (int q = 0; q < kMaxQ; ++q)
             if (q < nq) out[sub + 8 * q] = o[q];

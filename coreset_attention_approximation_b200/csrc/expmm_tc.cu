@@ -95,7 +95,7 @@ struct Smem {
     static constexpr uint32_t kTotal = Bar + 256;
     static constexpr uint32_t kAlloc = kTotal;          // the base is 1024-aligned (checked in the kernel)
     static_assert(kAlloc <= 232448, "shared memory per block");
-    static_assert(BM * (DV + 4) * 4 <= NC * kC, "the epilogue stages O in the value ring");
+    static_assert(BM * c1_row(DV) * 4 <= NC * kC, "the epilogue stages O in the value ring");
 };
 
 // TMEM: S / P buffer b (b = key block % 3) at columns 128 b .. +127 (P as
@@ -454,6 +454,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // T == 0) knows the final reference.  The other hands it log2 of its
         // share of the normaliser in its own reference; the last one adds the
         // two in the final reference and hands the total back.
+        // the column scales of the attention output, loaded before the waits below
+        float sgv[MODE == kExpmmRownorm ? DV / 2 : 1];
+        if (MODE == kExpmmRownorm) {
+            const float4* s4 = reinterpret_cast<const float4*>(args.sigma + (size_t)unit * DV + par * (DV / 2));
+#pragma unroll
+            for (int c = 0; c < DV / 2; c += 4) {
+                const float4 f = __ldg(s4 + c / 4);
+                sgv[c] = f.x;
+                sgv[c + 1] = f.y;
+                sgv[c + 2] = f.z;
+                sgv[c + 3] = f.w;
+            }
+        }
         const bool last = par == ((T + 1) & 1);
         float* tl = tok + BM;                   // second slot: only the epilogue uses it
         float lt;
@@ -476,17 +489,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) tc_fence_after();
         }
         // O goes out through shared memory (the value ring is idle once PV(T - 1)
-        // has completed): each warp stages half of the columns of its 32 rows,
-        // then the 256 softmax threads copy the block's rows, which are
-        // contiguous in global memory, with coalesced stores.
-        constexpr int SST = (MODE != kExpmmRownorm) ? DV + 2 : DV + 4;   // staged row stride (floats)
+        // has completed): each warp stages half of the columns of its 32 rows
+        // (staged rows DV + 4 floats apart, 16-byte aligned), then bulk
+        // asynchronous copies move the rows to global memory: the partial sums'
+        // rows are one contiguous run (the same row stride), attention rows go
+        // one copy per row.
+        constexpr int SST = c1_row(DV);
         float* stg = reinterpret_cast<float*>(sm + L::C0);
         const bool have_o = ok && T > 0;
         const uint32_t tO = tO0 + lanes + par * (DV / 2);
-        const int cbase = par * (DV / 2);
-        const float* sg = args.sigma + (size_t)unit * DV;
         const float inv = 1.f / lt;
-        float* srow = stg + row * SST + cbase;
+        float* srow = stg + row * SST + par * (DV / 2);
 #pragma unroll
         for (int c0 = 0; c0 < DV / 2; c0 += 32) {
             float o[32];
@@ -497,41 +510,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0.f;
             }
-            if (MODE != kExpmmRownorm) {
-                // staged rows are DV + 2 floats apart (the global layout): 8-byte aligned
 #pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    *reinterpret_cast<float2*>(srow + c0 + c) = make_float2(o[c], o[c + 1]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const int cc = cbase + c0 + c;
-                    *reinterpret_cast<float4*>(srow + c0 + c) =
-                        make_float4(o[c] * sg[cc] * inv, o[c + 1] * sg[cc + 1] * inv, o[c + 2] * sg[cc + 2] * inv,
-                                    o[c + 3] * sg[cc + 3] * inv);
+            for (int c = 0; c < 32; c += 4) {
+                float4 v = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                if (MODE == kExpmmRownorm) {
+                    v.x *= sgv[c0 + c] * inv;
+                    v.y *= sgv[c0 + c + 1] * inv;
+                    v.z *= sgv[c0 + c + 2] * inv;
+                    v.w *= sgv[c0 + c + 3] * inv;
                 }
+                *reinterpret_cast<float4*>(srow + c0 + c) = v;
             }
         }
         if (MODE != kExpmmRownorm && last) *reinterpret_cast<float2*>(stg + row * SST + DV) = make_float2(lt, mO * kLn2);
+        fence_async_smem();                     // the bulk copies read the staged rows through the async proxy
         softmax_sync();                         // all 8 softmax warps have staged their part
         const int rows = min(BM, a_valid - a0);
         const int st = tid - 4 * 32;            // 0 .. 255
-        if (ok) {
-            if (MODE != kExpmmRownorm) {
-                // rows a0 .. of this split are one contiguous run of rows * (DV + 2) floats
-                float2* dst = reinterpret_cast<float2*>(static_cast<float*>(args.out) +
-                                                        (((size_t)unit * args.nsplit + split) * args.r + a0) * (DV + 2));
-                const float2* src = reinterpret_cast<const float2*>(stg);
-                const int n2 = rows * (DV + 2) / 2;
-                for (int i = st; i < n2; i += 256) dst[i] = src[i];
-            } else {
-                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a0) * DV);
-                const int n4 = rows * (DV / 4);
-                for (int i = st; i < n4; i += 256) {
-                    const int rr = i / (DV / 4), c4 = i - rr * (DV / 4);
-                    dst[i] = *reinterpret_cast<const float4*>(stg + rr * SST + 4 * c4);
-                }
-            }
+        if (ok && MODE != kExpmmRownorm && st == 0) {
+            bulk_store(static_cast<float*>(args.out) + (((size_t)unit * args.nsplit + split) * args.r + a0) * SST, stg,
+                       (uint32_t)(rows * SST * 4));
+            bulk_commit();
+            bulk_wait_read_all();
+        }
+        if (ok && MODE == kExpmmRownorm && st < rows) {
+            bulk_store(static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a0 + st) * DV, stg + st * SST,
+                       (uint32_t)(DV * 4));
+            bulk_commit();
+            bulk_wait_read_all();
         }
     }
 
@@ -548,27 +554,56 @@ __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __
 }
 
 // Weights for the attention GEMM: per unit and column c < dv, sigma_c =
-// max_s |W[s, c]| and W16[s, c] = W[s, c] / sigma_c (fp16); wn[s] = W[s, dv]
-// padded with zeros to r_pad rows.  One block per unit.
-__global__ void weights_prep_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, __half* W16,
-                                    float* sigma, float* wn, int r, int r_pad, int dv, int all_keys) {
-    const int u = blockIdx.x;
+// max_s |W[s, c]| (1 if the column is zero), W16[s, c] = W[s, c] / sigma_c
+// (fp16) and wn[s] = W[s, dv], zero-padded to r_pad rows.  Rows >= the
+// unit's rank are zero (all r rows count with `all_keys`).
+// Column maxima: block (unit, 32 columns), 8 row groups of 32 threads.
+__global__ void weights_sigma_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, float* sigma,
+                                     int r, int dv, int all_keys) {
+    const int u = blockIdx.x, c = blockIdx.y * 32 + (threadIdx.x & 31), g = threadIdx.x >> 5;
     const int k = all_keys ? r : rank[u];
     const float* Wu = W + (size_t)u * r * (dv + 1);
-    __shared__ float sg[256];
-    for (int c = threadIdx.x; c < dv; c += blockDim.x) {
-        float mx = 0.f;
-        for (int s = 0; s < k; ++s) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
-        sg[c] = mx > 0.f ? mx : 1.f;
-        sigma[(size_t)u * dv + c] = sg[c];
-    }
+    float mx = 0.f;
+    if (c < dv)
+        for (int s = g; s < k; s += 8) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
+    __shared__ float part[8][32];
+    part[g][threadIdx.x & 31] = mx;
     __syncthreads();
-    for (int e = threadIdx.x; e < r * dv; e += blockDim.x) {
-        const int s = e / dv, c = e % dv;
-        const float v = s < k ? Wu[(size_t)s * (dv + 1) + c] / sg[c] : 0.f;
-        W16[(size_t)u * r * dv + e] = __float2half_rn(v);
+    if (g == 0 && c < dv) {
+        float m = part[0][threadIdx.x];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, part[i][threadIdx.x]);
+        sigma[(size_t)u * dv + c] = m > 0.f ? m : 1.f;
     }
-    for (int s = threadIdx.x; s < r_pad; s += blockDim.x) wn[(size_t)u * r_pad + s] = s < k ? Wu[(size_t)s * (dv + 1) + dv] : 0.f;
+}
+
+// The scaled fp16 weights and the normaliser column, grid-stride over every unit.
+__global__ void weights_half_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank,
+                                    const float* __restrict__ sigma, __half* W16, float* wn, int units, int r,
+                                    int r_pad, int dv, int all_keys) {
+    const size_t per = (size_t)r * dv, total = (size_t)units * per;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+        const int u = (int)(e / per);
+        const int rem = (int)(e - (size_t)u * per);
+        const int s = rem / dv, c = rem - s * dv;
+        const int k = all_keys ? r : rank[u];
+        const float v = s < k ? W[((size_t)u * r + s) * (dv + 1) + c] / sigma[(size_t)u * dv + c] : 0.f;
+        W16[e] = __float2half_rn(v);
+    }
+    const size_t tw = (size_t)units * r_pad;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < tw; e += (size_t)gridDim.x * blockDim.x) {
+        const int u = (int)(e / r_pad), s = (int)(e - (size_t)u * r_pad);
+        const int k = all_keys ? r : rank[u];
+        wn[e] = s < k ? W[((size_t)u * r + s) * (dv + 1) + dv] : 0.f;
+    }
+}
+
+wc_status launch_weights_prep(const Shape& s, const float* W, const int32_t* rank, __half* W16, float* sigma,
+                              float* wn, cudaStream_t st) {
+    weights_sigma_kernel<<<dim3(s.units, (s.dv + 31) / 32), 256, 0, st>>>(W, rank, sigma, s.r, s.dv, s.bins > 1);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    weights_half_kernel<<<1184, 256, 0, st>>>(W, rank, sigma, W16, wn, s.units, s.r, s.r_pad, s.dv, s.bins > 1);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -669,8 +704,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     __half* W16 = reinterpret_cast<__half*>(ws + Lw.w16);
     float* sigma = reinterpret_cast<float*>(ws + Lw.sigma);
     float* wn = reinterpret_cast<float*>(ws + Lw.wn);
-    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv, s.bins > 1);
-    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    if (launch_weights_prep(s, W, rank, W16, sigma, wn, st) != WC_OK) return WC_ERR_CUDA;
     CUtensorMap mA, mB, mC;
     if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
         !make_map(&mB, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BN) ||
@@ -702,8 +736,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
 // point that allocates nothing.
 wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
                               float* out, int* status, __half* W16, float* sigma, float* wn, cudaStream_t st) {
-    weights_prep_kernel<<<s.units, 256, 0, st>>>(W, rank, W16, sigma, wn, s.r, s.r_pad, s.dv, s.bins > 1);
-    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+    if (launch_weights_prep(s, W, rank, W16, sigma, wn, st) != WC_OK) return WC_ERR_CUDA;
     CUtensorMap mA, mB, mC;
     if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
         !make_map(&mB, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BN) ||

@@ -13,6 +13,8 @@ namespace wc {
 constexpr int kMaxBlocksPerUnit = 512;   // select: thread blocks that share one unit
 constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1
 constexpr int kCenterChunk = 1024;       // centring: keys per partial column sum
+// Row of a C1 partial sum: O[0 .. dv), l, m, two unused floats (rows 16-byte aligned).
+constexpr int c1_row(int dv) { return dv + 4; }
 constexpr int kWsAlign = 256;
 
 // One per unit, in the workspace; zeroed before every select launch.
@@ -34,7 +36,7 @@ struct WsLayout {
     size_t partials;  // double[units][2][kMaxBlocksPerUnit]
     size_t kt;        // dtype[units][d][ldf]   transposed keys
     size_t lg;        // float[units][r][r]     gathered L = F[piv, :]
-    size_t c1part;    // float[units][nsplit][r][dv + 2]  (O | l | m)
+    size_t c1part;    // float[units][nsplit][r][c1_row(dv)]  (O | l | m | unused)
     size_t y;         // double[units][dv + 1][r]  C1, column-major, solved in place
     size_t v16;       // half[units][n][dv]     values for the tensor-core weights GEMM
     size_t w16;       // half[units][r][dv]     column-scaled weights for attention

@@ -54,7 +54,7 @@ __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t*
         const int uc = u / bins;  // the caller's unit
         rho = beta * (kk[uc] - cdot[(size_t)uc * n_all + piv[(size_t)u * r + a]]);
     }
-    const int w = dv + 2, wcols = dv + 1;
+    const int w = c1_row(dv), wcols = dv + 1;
     const float* part = c1part + (size_t)u * nsplit * r * w;
     double mx = -INFINITY;
     for (int sp = 0; sp < nsplit; ++sp) mx = fmax(mx, (double)part[((size_t)sp * r + a) * w + dv + 1]);
