@@ -11,7 +11,9 @@ namespace wc {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-static int64_t f_ld(int32_t n) { return ((int64_t)n + 7) / 8 * 8; }
+// Row stride of F (and of the transposed keys): n rounded up to 64 elements, so
+// every row of F starts on a 256-byte boundary.
+static int64_t f_ld(int32_t n) { return ((int64_t)n + 63) / 64 * 64; }
 
 wc_status make_shape(const wc_shape* in, Shape* o) {
     if (!in) return WC_ERR_INVALID;

@@ -33,7 +33,16 @@ namespace wc {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kGroup = 8;  // rows per thread per pass (two float4 of F)
+// rows per thread per pass (one float2 of F): with about 14 rows of a block's
+// slice per thread, 2-row groups keep the threads of a block evenly loaded
+// (8-row groups left a seventh of a step idle), and the streams go as 8-byte
+// loads, 32 of them in flight per thread
+constexpr int kGroup = 2;
+// Rows per block are a multiple of 128, so every block's slice of F (fp32) and
+// of the transposed keys (bf16) starts on a 256-byte boundary: blocks whose
+// slices did not streamed their share about 6 % slower, and every step waits
+// for the slowest block of the unit.
+constexpr int kRowAlign = 128;
 
 struct SelectArgs {
     const void* K;
@@ -47,7 +56,7 @@ struct SelectArgs {
     int64_t ldf;
     int32_t n, d, r;
     int32_t C;      // blocks per unit
-    int32_t m;      // rows per block (multiple of kGroup)
+    int32_t m;      // rows per block (multiple of kRowAlign)
     int32_t unit0;  // first unit of this wave
     double beta, eps;
     uint64_t seed;
@@ -61,6 +70,7 @@ struct SelectArgs {
 __host__ __device__ inline size_t select_smem_bytes(int m, int r, int d) {
     return (size_t)m * 8          // residual diagonal (fp64)
            + (size_t)kThreads * 8 // per-thread inclusive scan
+           + (size_t)kMaxBlocksPerUnit * 8  // the unit's block sums of a step
            + (size_t)d * 8        // pivot key
            + (size_t)r * 4        // F[s, 0..j)
            + (size_t)m            // pivot flags
@@ -109,96 +119,103 @@ __device__ __forceinline__ void chunk_of(int t, int mlen, int* lo, int* hi) {
     *hi = min(mlen, *lo + q);
 }
 
-__device__ __forceinline__ void unpack_bf16x8(uint4 raw, float x[8]) {
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        x[2 * k] = __uint_as_float(w[k] << 16);
-        x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
+__device__ __forceinline__ float2 ld_stream_f2(const float* p) {
+    float2 v;
+    asm volatile("ld.global.L1::no_allocate.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+    return v;
 }
 
-// <k_i, k_s> for the 8 rows at Kt + i0 (column stride ldf).
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// <k_i, k_s> for the 2 rows at Kt + i0 (column stride ldf): products of 8
+// consecutive dimensions summed in fp32, the chunks summed in fp64.
 template <typename T>
-__device__ __forceinline__ void key_dots(const T* Kt, int64_t ldf, int d, const double* ks, double dot[8]);
+__device__ __forceinline__ void key_dots(const T* Kt, int64_t ldf, int d, const double* ks, double dot[2]);
 
 template <>
 __device__ __forceinline__ void key_dots<__nv_bfloat16>(const __nv_bfloat16* Kt, int64_t ldf, int d,
-                                                       const double* ks, double dot[8]) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) dot[k] = 0.0;
+                                                       const double* ks, double dot[2]) {
+    dot[0] = dot[1] = 0.0;
+#pragma unroll 4
     for (int c0 = 0; c0 < d; c0 += 8) {
-        float acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            float x[8];
-            unpack_bf16x8(ld_stream_u4(Kt + (int64_t)(c0 + c) * ldf), x);
+            const uint32_t w = ld_stream_u32(Kt + (int64_t)(c0 + c) * ldf);
             const float kc = (float)ks[c0 + c];  // exact: ks holds bf16 values
-#pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = fmaf(x[k], kc, acc[k]);
+            a0 = fmaf(__uint_as_float(w << 16), kc, a0);
+            a1 = fmaf(__uint_as_float(w & 0xffff0000u), kc, a1);
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) dot[k] += (double)acc[k];
+        dot[0] += (double)a0;
+        dot[1] += (double)a1;
     }
 }
 
 template <>
 __device__ __forceinline__ void key_dots<float>(const float* Kt, int64_t ldf, int d, const double* ks,
-                                               double dot[8]) {
-    // fp32 inputs: products and sums in fp64
-#pragma unroll
-    for (int k = 0; k < 8; ++k) dot[k] = 0.0;
+                                               double dot[2]) {
+    // fp32 (or centred) keys: products and sums in fp64
+    dot[0] = dot[1] = 0.0;
+#pragma unroll 8
     for (int c = 0; c < d; ++c) {
-        const float4 a = ld_stream_f4(Kt + (int64_t)c * ldf);
-        const float4 b = ld_stream_f4(Kt + (int64_t)c * ldf + 4);
+        const float2 v = ld_stream_f2(Kt + (int64_t)c * ldf);
         const double kc = ks[c];
-        dot[0] += (double)a.x * kc; dot[1] += (double)a.y * kc;
-        dot[2] += (double)a.z * kc; dot[3] += (double)a.w * kc;
-        dot[4] += (double)b.x * kc; dot[5] += (double)b.y * kc;
-        dot[6] += (double)b.z * kc; dot[7] += (double)b.w * kc;
+        dot[0] += (double)v.x * kc;
+        dot[1] += (double)v.y * kc;
     }
 }
 
-// sum_{c<j} F[c, i] F[c, s] for the 8 rows at Fi (column stride ldf).
-__device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, const float* fs,
-                                           double cor[8]) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) cor[k] = 0.0;
+// sum_{c<j} F[c, i] F[c, s] for the 2 rows at Fi (column stride ldf): products
+// of 8 consecutive columns summed in fp32, the chunks summed in fp64.  32
+// columns are loaded before any is used.
+__device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, const float* fs, double cor[2]) {
+    cor[0] = cor[1] = 0.0;
     int c0 = 0;
-    for (; c0 + 8 <= j; c0 += 8) {
-        float acc[8];
+    for (; c0 + 32 <= j; c0 += 32) {
+        float2 v[32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        for (int c = 0; c < 32; ++c) v[c] = ld_stream_f2(Fi + (int64_t)(c0 + c) * ldf);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 f0 = *reinterpret_cast<const float4*>(fs + c0 + 8 * q);
+            const float4 f1 = *reinterpret_cast<const float4*>(fs + c0 + 8 * q + 4);
+            const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                a0 = fmaf(v[8 * q + c].x, f[c], a0);
+                a1 = fmaf(v[8 * q + c].y, f[c], a1);
+            }
+            cor[0] += (double)a0;
+            cor[1] += (double)a1;
+        }
+    }
+    for (; c0 + 8 <= j; c0 += 8) {
+        float2 v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[c] = ld_stream_f2(Fi + (int64_t)(c0 + c) * ldf);
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const float* p = Fi + (int64_t)(c0 + c) * ldf;
-            const float4 a = ld_stream_f4(p), b = ld_stream_f4(p + 4);
-            const float f = fs[c0 + c];
-            acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
-            acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
-            acc[4] = fmaf(b.x, f, acc[4]); acc[5] = fmaf(b.y, f, acc[5]);
-            acc[6] = fmaf(b.z, f, acc[6]); acc[7] = fmaf(b.w, f, acc[7]);
+            a0 = fmaf(v[c].x, fs[c0 + c], a0);
+            a1 = fmaf(v[c].y, fs[c0 + c], a1);
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) cor[k] += (double)acc[k];
+        cor[0] += (double)a0;
+        cor[1] += (double)a1;
     }
     if (c0 < j) {
-        float acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        float a0 = 0.f, a1 = 0.f;
         for (int c = c0; c < j; ++c) {
-            const float* p = Fi + (int64_t)c * ldf;
-            const float4 a = ld_stream_f4(p), b = ld_stream_f4(p + 4);
-            const float f = fs[c];
-            acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
-            acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
-            acc[4] = fmaf(b.x, f, acc[4]); acc[5] = fmaf(b.y, f, acc[5]);
-            acc[6] = fmaf(b.z, f, acc[6]); acc[7] = fmaf(b.w, f, acc[7]);
+            const float2 v = ld_stream_f2(Fi + (int64_t)c * ldf);
+            a0 = fmaf(v.x, fs[c], a0);
+            a1 = fmaf(v.y, fs[c], a1);
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) cor[k] += (double)acc[k];
+        cor[0] += (double)a0;
+        cor[1] += (double)a1;
     }
 }
 
@@ -215,11 +232,14 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     const int r0 = min(n, blk * a.m);
     const int r1 = min(n, r0 + a.m);
     const int mlen = r1 - r0;
-    const int ng = (mlen + kGroup - 1) / kGroup;
+    // groups this block computes: its rows, and for the last block the padding
+    // up to the row stride ldf as well (F is zero there)
+    const int ng = r1 == n ? (int)((ldf - r0 + kGroup - 1) / kGroup) : (mlen + kGroup - 1) / kGroup;
 
     double* dg = reinterpret_cast<double*>(smem);
     double* scan = dg + a.m;
-    double* ks = scan + kThreads;
+    double* bsum = scan + kThreads;
+    double* ks = bsum + kMaxBlocksPerUnit;
     float* fs = reinterpret_cast<float*>(ks + d);
     unsigned char* ispiv = reinterpret_cast<unsigned char*>(fs + r);
     __shared__ Bcast bc;
@@ -252,9 +272,9 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             lmax = fmax(lmax, dg[il]);
         } else {
             for (int c = 0; c < d; ++c) Kt[(int64_t)c * ldf + i] = TK(0.f);
-            dg[il] = 0.0;
+            if (il < a.m) dg[il] = 0.0;
         }
-        ispiv[il] = 0;
+        if (il < a.m) ispiv[il] = 0;
     }
     // block max of H_ii -> unit max (positive doubles order like their bits)
 #pragma unroll
@@ -283,10 +303,14 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     int final_rank = alive ? r : 0;
     for (int j = 0; alive && j < r; ++j) {
         const double* pj = part + (size_t)(j & 1) * kMaxBlocksPerUnit;
-        // 1. which block's slice holds t = u_j * sum(d)
+        // 1. which block's slice holds t = u_j * sum(d): the unit's block sums
+        // come into shared memory in parallel, then one thread adds them in
+        // block order
+        for (int c = tid; c < a.C; c += kThreads) bsum[c] = __ldcg(pj + c);
+        __syncthreads();
         if (tid == 0) {
             double total = 0.0;
-            for (int c = 0; c < a.C; ++c) total += __ldcg(pj + c);
+            for (int c = 0; c < a.C; ++c) total += bsum[c];
             bc.stop = 0;
             bc.owner = -1;
             if (!(total > 0.0)) {
@@ -296,14 +320,14 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
                 const double tau = pivot_uniform(a.seed, (uint32_t)j, (uint32_t)unit) * total;
                 double run = 0.0;
                 for (int c = 0; c < a.C; ++c) {
-                    const double nxt = run + __ldcg(pj + c);
+                    const double nxt = run + bsum[c];
                     if (nxt > tau) { bc.owner = c; bc.base = run; break; }
                     run = nxt;
                 }
                 if (bc.owner < 0) {  // rounding left tau at the top: last block with mass
                     run = 0.0;
                     for (int c = 0; c < a.C; ++c) {
-                        const double p = __ldcg(pj + c);
+                        const double p = bsum[c];
                         if (p > 0.0) { bc.owner = c; bc.base = run; }
                         run += p;
                     }
@@ -368,7 +392,17 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
 
         // 3. pivot key and F[s, 0..j) into shared memory
         for (int c = tid; c < d; c += kThreads) ks[c] = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
-        for (int c = tid; c < j; c += kThreads) fs[c] = ld_cg_f32(F + (int64_t)c * ldf + s);
+        for (int c0 = tid; c0 < j; c0 += 8 * kThreads) {  // 8 loads in flight before the stores
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int c = c0 + q * kThreads;
+                v[q] = c < j ? ld_cg_f32(F + (int64_t)c * ldf + s) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (c0 + q * kThreads < j) fs[c0 + q * kThreads] = v[q];
+        }
         __syncthreads();
 
         // 4. column j over this block's rows, and the residual downdate
@@ -377,12 +411,12 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         for (int g = tid; g < ng; g += kThreads) {
             const int il0 = g * kGroup;
             const int i0 = r0 + il0;
-            double dot[8], cor[8];
+            double dot[kGroup], cor[kGroup];
             key_dots<TK>(Kt + i0, ldf, d, ks, dot);
             correction(F + i0, ldf, j, fs, cor);
-            float out[8];
+            float out[kGroup];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < kGroup; ++k) {
                 const int il = il0 + k;
                 double f = 0.0;
                 if (il < mlen && !ispiv[il]) f = (exp(a.beta * dot[k]) - cor[k]) / root;
@@ -392,8 +426,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
                     dg[il] = nd > 0.0 ? nd : 0.0;
                 }
             }
-            *reinterpret_cast<float4*>(Fj + i0) = make_float4(out[0], out[1], out[2], out[3]);
-            *reinterpret_cast<float4*>(Fj + i0 + 4) = make_float4(out[4], out[5], out[6], out[7]);
+            *reinterpret_cast<float2*>(Fj + i0) = make_float2(out[0], out[1]);
         }
         __syncthreads();
         if (s >= r0 && s < r1 && tid == 0) {
@@ -423,8 +456,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         float* Fj = F + (int64_t)jj * ldf;
         for (int g = tid; g < ng; g += kThreads) {
             const int i0 = r0 + g * kGroup;
-            *reinterpret_cast<float4*>(Fj + i0) = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(Fj + i0 + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float2*>(Fj + i0) = make_float2(0.f, 0.f);
         }
     }
     if (blk == 0) {
@@ -446,7 +478,7 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     // rows per block bounded by shared memory (fp64 diagonal + flags)
     const size_t fixed = select_smem_bytes(0, s.r, s.d) + 1024;
     if ((size_t)max_smem <= fixed) return WC_ERR_UNSUPPORTED;
-    int m_max = (int)(((size_t)max_smem - fixed) / 9) / kGroup * kGroup;
+    int m_max = (int)(((size_t)max_smem - fixed) / 9) / kRowAlign * kRowAlign;
     m_max = m_max > (1 << 20) ? (1 << 20) : m_max;
 
     auto kern = rpcholesky_kernel<T, TK>;
@@ -459,7 +491,7 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
             return 0;
         return b;
     };
-    auto rows_for = [&](int C) { return ((s.n + C - 1) / C + kGroup - 1) / kGroup * kGroup; };
+    auto rows_for = [&](int C) { return ((s.n + C - 1) / C + kRowAlign - 1) / kRowAlign * kRowAlign; };
 
     // Most blocks per unit such that every block of the launch is co-resident
     // (they wait on each other), at >= 256 rows per block; else the fewest

@@ -111,7 +111,7 @@ typedef struct {
                          before the selection and the weights; see "Centring" above */
 } wc_shape;
 
-/* Row stride (elements) of F for n_k keys: n_k rounded up to a multiple of 8. */
+/* Row stride (elements) of F for n_k keys: n_k rounded up to a multiple of 64. */
 int64_t wc_f_ld(int32_t n_k);
 
 /* Workspace bytes that select, weights, attend and forward need for `shape`

@@ -53,8 +53,8 @@ def test_status_strings(lib):
     assert lib.wc_status_string(99) == b"unknown status"
 
 
-def test_f_ld_rounds_to_eight(lib):
-    assert [wildcat.f_ld(n) for n in (1, 7, 8, 9, 1000, 131072)] == [8, 8, 8, 16, 1000, 131072]
+def test_f_ld_rounds_to_sixty_four(lib):
+    assert [wildcat.f_ld(n) for n in (1, 63, 64, 65, 1000, 131072)] == [64, 64, 64, 128, 1024, 131072]
 
 
 def test_workspace_sizes(lib):
