@@ -114,3 +114,36 @@ def test_center_changes_the_selection_but_not_exactness():
     b = run_gpu(Q, K, V, w.r, seed=4)
     assert not torch.equal(a["piv"], b["piv"])
     compare_next(Q, K, V, w.r, seed=4, center=True, tol_w=2e-3)
+
+
+def test_bins_without_queries_runs_select_and_weights():
+    w = WORKLOADS["vit"].replace(batch=1, hq=2, hkv=2, n_q=0)
+    Q, K, V = make_inputs(w)
+    res = run_gpu(Q, K, V, w.r, seed=7, bins=4)
+    assert res["rank"].shape == (1, 2, 4) and np.all(res["rank"].numpy() == w.r // 4)
+    assert res["out"].numel() == 0
+
+
+def test_bins_one_pivot_per_bin():
+    w = WORKLOADS["vit"].replace(batch=1, hq=2, hkv=2, n_k=512, n_q=40, r=8)
+    compare_next(*make_inputs(w, seed=8), 8, seed=8, bins=8, tol_w=2e-3)
+
+
+def test_center_with_bins_fp32():
+    w = WORKLOADS["tiny"]
+    compare_next(*_offset(w, 9, 0.4), w.r, seed=9, bins=4, center=True, tol_w=1e-5)
+
+
+def test_bins_attend_without_allocation():
+    # the attention entry that allocates nothing takes every union row as well
+    from coreset_attention_approximation_b200 import wildcat
+    w = WORKLOADS["diffusion"].replace(batch=1, hq=2, hkv=2, n_k=2048, n_q=300, r=128)
+    Q, K, V = [t.cuda() for t in make_inputs(w, seed=11)]
+    res = wildcat.forward(Q, K, V, w.r, seed=11, bins=4)
+    want = wildcat.attend(Q, res["Ks"], res["W"], res["rank"], w.n_k, bins=4)
+    got = wildcat.attend_noalloc(Q, res["Ks"], res["W"], res["rank"], w.n_k, bins=4)
+    torch.cuda.synchronize()
+    assert wildcat.check_device_status(res["ws"]) == 0
+    for h in range(w.hq):
+        assert rel_err(got[0, h].cpu().numpy(), want[0, h].cpu().numpy()) <= TOL_OUT[torch.bfloat16]
+        assert rel_err(got[0, h].cpu().numpy(), res["out"][0, h].cpu().numpy()) <= TOL_OUT[torch.bfloat16]
