@@ -105,23 +105,6 @@ __device__ __forceinline__ double pivot_uniform(uint64_t seed, uint32_t j, uint3
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// 16-byte load that does not allocate in L1 (each line is used once per pass).
-__device__ __forceinline__ float4 ld_stream_f4(const float* p) {
-    float4 v;
-    asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 // Load that bypasses L1 (data another block wrote during this launch).
 __device__ __forceinline__ float ld_cg_f32(const float* p) { return __ldcg(p); }
 
