@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
                                                            const double* __restrict__ Ct, float* W, int r, int dv) {
     extern __shared__ double sm_d[];
     double* Y = sm_d;                                        // [r][NC]
-    float* Ld = reinterpret_cast<float*>(Y + (size_t)r * NC);  // [kTB][kTB + 1] diagonal block
+    double* rinv = Y + (size_t)r * NC;                       // [kTB] 1 / L_ii of the diagonal block
+    float* Ld = reinterpret_cast<float*>(rinv + kTB);        // [kTB][kTB + 1] diagonal block
     const int u = blockIdx.y;
     const int wcols = dv + 1;
     const int c0 = blockIdx.x * NC;
@@ -101,28 +102,35 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
     const double* C = Ct + (size_t)u * wcols * r;
     float* Wu = W + (size_t)u * r * wcols;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool rows16 = (r & 3) == 0;  // rows of L start on 16-byte boundaries
 
     for (int e = tid; e < NC * k; e += kTrsmThreads) {
         const int q = e / k, a = e - q * k;
         Y[a * NC + q] = q < nc ? C[(size_t)(c0 + q) * r + a] : 0.0;
     }
 
-    // ---- forward: L y = c
-    for (int kb = 0; kb < k; kb += kTB) {
-        const int bs = min(kTB, k - kb);
+    // The diagonal block [kb, kb + bs) of L into shared memory, with 1 / L_ii.
+    auto stage_diag = [&](int kb, int bs) {
         __syncthreads();
         for (int e = tid; e < kTB * kTB; e += kTrsmThreads) {
             const int i = e / kTB, j = e % kTB;
             Ld[i * (kTB + 1) + j] = (i < bs && j <= i) ? L[(size_t)(kb + i) * r + kb + j] : 0.f;
         }
+        if (tid < kTB) rinv[tid] = tid < bs ? 1.0 / (double)L[(size_t)(kb + tid) * r + kb + tid] : 0.0;
         __syncthreads();
+    };
+
+    // ---- forward: L y = c
+    for (int kb = 0; kb < k; kb += kTB) {
+        const int bs = min(kTB, k - kb);
+        stage_diag(kb, bs);
         if (warp < NC) {
             const int q = warp;
             double y0 = lane < bs ? Y[(kb + lane) * NC + q] : 0.0;
             double y1 = lane + 32 < bs ? Y[(kb + lane + 32) * NC + q] : 0.0;
             for (int i = 0; i < bs; ++i) {
                 const double own = (i < 32) ? y0 : y1;
-                const double yi = __shfl_sync(0xffffffffu, own / (double)Ld[i * (kTB + 1) + i], i & 31);
+                const double yi = __shfl_sync(0xffffffffu, own * rinv[i], i & 31);
                 if (lane == (i & 31)) {
                     if (i < 32) y0 = yi;
                     else y1 = yi;
@@ -134,15 +142,30 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
             if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
         }
         __syncthreads();
+        // every later row i: Y_i -= L[i, kb .. kb + bs) Y[kb .. kb + bs), 8 entries of L in flight
         for (int i = kb + bs + tid; i < k; i += kTrsmThreads) {
             double acc[NC];
 #pragma unroll
             for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
             const float* Li = L + (size_t)i * r + kb;
-            for (int b = 0; b < bs; ++b) {
-                const double l = (double)Li[b];
+            for (int b0 = 0; b0 < bs; b0 += 8) {
+                float lv[8];
+                if (rows16 && b0 + 8 <= bs) {
+                    const float4 x = __ldg(reinterpret_cast<const float4*>(Li + b0));
+                    const float4 y = __ldg(reinterpret_cast<const float4*>(Li + b0 + 4));
+                    lv[0] = x.x; lv[1] = x.y; lv[2] = x.z; lv[3] = x.w;
+                    lv[4] = y.x; lv[5] = y.y; lv[6] = y.z; lv[7] = y.w;
+                } else {
 #pragma unroll
-                for (int q = 0; q < NC; ++q) acc[q] -= l * Y[(kb + b) * NC + q];
+                    for (int e = 0; e < 8; ++e) lv[e] = b0 + e < bs ? __ldg(Li + b0 + e) : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const double l = (double)lv[e];
+                    const double* yb = Y + (kb + b0 + e) * NC;
+#pragma unroll
+                    for (int q = 0; q < NC; ++q) acc[q] -= l * yb[q];
+                }
             }
 #pragma unroll
             for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
@@ -152,19 +175,14 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
     // ---- backward: L^T x = y
     for (int kb = (k - 1) / kTB * kTB; k > 0 && kb >= 0; kb -= kTB) {
         const int bs = min(kTB, k - kb);
-        __syncthreads();
-        for (int e = tid; e < kTB * kTB; e += kTrsmThreads) {
-            const int i = e / kTB, j = e % kTB;
-            Ld[i * (kTB + 1) + j] = (i < bs && j <= i) ? L[(size_t)(kb + i) * r + kb + j] : 0.f;
-        }
-        __syncthreads();
+        stage_diag(kb, bs);
         if (warp < NC) {
             const int q = warp;
             double y0 = lane < bs ? Y[(kb + lane) * NC + q] : 0.0;
             double y1 = lane + 32 < bs ? Y[(kb + lane + 32) * NC + q] : 0.0;
             for (int i = bs - 1; i >= 0; --i) {
                 const double own = (i < 32) ? y0 : y1;
-                const double xi = __shfl_sync(0xffffffffu, own / (double)Ld[i * (kTB + 1) + i], i & 31);
+                const double xi = __shfl_sync(0xffffffffu, own * rinv[i], i & 31);
                 if (lane == (i & 31)) {
                     if (i < 32) y0 = xi;
                     else y1 = xi;
@@ -176,14 +194,22 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
             if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
         }
         __syncthreads();
+        // every earlier row i: Y_i -= L[kb .. kb + bs, i]^T Y[kb .. kb + bs) (loads coalesced across i)
         for (int i = tid; i < kb; i += kTrsmThreads) {
             double acc[NC];
 #pragma unroll
             for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
-            for (int b = 0; b < bs; ++b) {
-                const double l = (double)L[(size_t)(kb + b) * r + i];
+            for (int b0 = 0; b0 < bs; b0 += 8) {
+                float lv[8];
 #pragma unroll
-                for (int q = 0; q < NC; ++q) acc[q] -= l * Y[(kb + b) * NC + q];
+                for (int e = 0; e < 8; ++e) lv[e] = b0 + e < bs ? __ldg(L + (size_t)(kb + b0 + e) * r + i) : 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const double l = (double)lv[e];
+                    const double* yb = Y + (kb + b0 + e) * NC;
+#pragma unroll
+                    for (int q = 0; q < NC; ++q) acc[q] -= l * yb[q];
+                }
             }
 #pragma unroll
             for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
@@ -198,7 +224,7 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
 
 template <int NC>
 size_t trsm_smem(int r) {
-    return sizeof(double) * NC * (size_t)r + sizeof(float) * kTB * (kTB + 1);
+    return sizeof(double) * (NC * (size_t)r + kTB) + sizeof(float) * kTB * (kTB + 1);
 }
 
 template <int NC>
