@@ -363,9 +363,10 @@ def run_ours(args, world, rank, local):
     return res
 
 
-# select (1 cooperative wave here), gather, fp16 copy of V, C1 exp-GEMM, merge of
-# the C1 partials, triangular solves, weight scales, fp16 weights, attention exp-GEMM
-LAUNCHES_PER_STEP = 9
+# select (1 cooperative wave here), the factor's shift for the weights, gather, fp16
+# copy of V, C1 exp-GEMM, merge of the C1 partials, triangular solves, weight
+# scales, fp16 weights, attention exp-GEMM
+LAUNCHES_PER_STEP = 10
 # centring: column sums, mean, key-mean dots, once in the select and once in the weights
 CENTER_LAUNCHES = 6
 
@@ -392,7 +393,7 @@ def kernel_breakdown(step):
             short = "attend_gemm" if m.group(2) == "1" else "weights_gemm"  # modes 0, 2: weights; 1: attention
         else:
             for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
-                             ("merge_c1", "merge_c1"), ("trsm_kernel", "solve"), ("weights_sigma", "w_prep"), ("weights_half", "w_prep")):
+                             ("merge_c1", "merge_c1"), ("trsm_kernel", "solve"), ("weights_sigma", "w_prep"), ("weights_half", "w_prep"), ("key_shift", "shift")):
                 if key in name:
                     short = tag
                     break

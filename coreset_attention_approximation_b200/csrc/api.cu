@@ -98,6 +98,7 @@ WsLayout make_layout(const Shape& s) {
     L.kk = take(C * sizeof(double) * U);
     L.cdot = take(C * sizeof(double) * U * n);
     L.bias = take(C * sizeof(float) * U * B * ((nb + 127) / 128 * 128));
+    L.shift = take(sizeof(double) * U * B);
     L.scratch_end = off;
     L.piv = take(sizeof(int32_t) * U * r);
     L.rank = take(sizeof(int32_t) * U * B);
@@ -162,6 +163,7 @@ wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Shape sb = bin_view(s);
     if (s.center && (e = launch_center(s, K, w, st)) != WC_OK) return e;
+    if ((e = launch_key_shift(s, K, w, st)) != WC_OK) return e;
     if ((e = launch_gather(sb, K, piv, F, rank, Ks, w, st)) != WC_OK) return e;
     if ((e = launch_coreset_values(sb, Ks, K, V, rank, w, st)) != WC_OK) return e;
     return launch_solve(sb, piv, rank, W, w, st);

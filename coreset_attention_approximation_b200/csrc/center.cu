@@ -1,4 +1,4 @@
-// center.cu — key centring statistics.
+// center.cu — key statistics: centring and the factor's shift.
 //
 // Method: WildCat: Near-Linear Attention in Theory and Practice (gist.science
 // technical summary, "Methodik" item 3): softmax attention is invariant to a
@@ -97,9 +97,57 @@ wc_status launch_center_t(const Shape& s, const void* K, char* ws, cudaStream_t 
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
+// M[u'] = max over bin unit u''s keys of beta |k_i|^2 (k_i - kbar when centred),
+// each |.|^2 summed in fp64 in dimension order as the selection sums it, so
+// the two agree bit for bit.  Blocks (chunk of kShiftChunk keys, bin unit);
+// the block maxima meet in an atomic maximum on the bits (non-negative doubles
+// order like their bits; a maximum is exact, so the result is deterministic).
+constexpr int kShiftChunk = 2048;
+
+template <typename T>
+__global__ void key_shift_kernel(const T* __restrict__ K, const double* __restrict__ kbar,
+                                 unsigned long long* shift_bits, int n, int d, int bins, double beta) {
+    const int ub = blockIdx.y;               // bin unit: caller unit ub / bins, bin ub % bins
+    const int nb = n / bins;
+    const T* Kb = K + (size_t)ub * nb * d;   // the bin's keys are contiguous
+    const double* m = kbar ? kbar + (size_t)(ub / bins) * d : nullptr;
+    const int i0 = blockIdx.x * kShiftChunk, i1 = min(nb, i0 + kShiftChunk);
+    double mx = 0.0;
+    for (int i = i0 + (int)threadIdx.x; i < i1; i += blockDim.x) {
+        const T* k = Kb + (size_t)i * d;
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) {
+            double x = (double)to_f32(k[c]);
+            if (m) x -= m[c];
+            ss += x * x;
+        }
+        mx = fmax(mx, beta * ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0 && mx > 0.0) atomicMax(shift_bits + ub, (unsigned long long)__double_as_longlong(mx));
+}
+
+template <typename T>
+wc_status launch_key_shift_t(const Shape& s, const void* K, char* ws, cudaStream_t st) {
+    const WsLayout L = make_layout(s);
+    const double* kbar = s.center ? reinterpret_cast<const double*>(ws + L.kbar) : nullptr;
+    const int ub = s.units_all * s.bins, nb = s.n_all / s.bins;
+    if (cudaMemsetAsync(ws + L.shift, 0, sizeof(double) * ub, st) != cudaSuccess) return WC_ERR_CUDA;
+    key_shift_kernel<T><<<dim3((nb + kShiftChunk - 1) / kShiftChunk, ub), 256, 0, st>>>(
+        static_cast<const T*>(K), kbar, reinterpret_cast<unsigned long long*>(ws + L.shift), s.n_all, s.d, s.bins,
+        s.beta);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
 }  // namespace
 
 int center_bias_stride(const Shape& s) { return (s.n_all / s.bins + 127) / 128 * 128; }
+
+wc_status launch_key_shift(const Shape& s, const void* K, char* ws, cudaStream_t st) {
+    if (s.dtype == WC_BF16) return launch_key_shift_t<__nv_bfloat16>(s, K, ws, st);
+    return launch_key_shift_t<float>(s, K, ws, st);
+}
 
 wc_status launch_center(const Shape& s, const void* K, char* ws, cudaStream_t st) {
     if (s.dtype == WC_BF16) return launch_center_t<__nv_bfloat16>(s, K, ws, st);

@@ -252,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     double* part = a.partials + (size_t)unit * 2 * kMaxBlocksPerUnit;
     int* status = a.status;
 
-    // ---- initial residual: d_i = H_ii = exp(beta |k_i|^2); transpose the slice
-    // (centred: k_i - kbar, in fp64 for the diagonal, stored as fp32)
+    // ---- initial residual in the log domain, beta |k_i|^2 (centred: k_i - kbar, in
+    // fp64, the transposed copy stored as fp32); transpose the slice
     double lmax = 0.0;
     for (int il = tid; il < ng * kGroup; il += kThreads) {
         const int i = r0 + il;
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
                 if constexpr (std::is_same<T, TK>::value) Kt[(int64_t)c * ldf + i] = kb ? TK((float)x) : v;
                 else Kt[(int64_t)c * ldf + i] = (TK)(float)x;
             }
-            dg[il] = exp(a.beta * ss);
+            dg[il] = a.beta * ss;
             lmax = fmax(lmax, dg[il]);
         } else {
             for (int c = 0; c < d; ++c) Kt[(int64_t)c * ldf + i] = TK(0.f);
@@ -276,12 +276,25 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         }
         if (il < a.m) ispiv[il] = 0;
     }
-    // block max of H_ii -> unit max (positive doubles order like their bits)
+    // block max of beta |k_i|^2 -> unit max M (non-negative doubles order like their bits)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
     if ((tid & 31) == 0 && lmax > 0.0) atomicMax(&us->hmax_bits, (unsigned long long)__double_as_longlong(lmax));
+    bool alive = unit_barrier(&us->bar, a.C, 1, a.timeout_ns, status, &bc.ok);
+    // The factor is taken of the shifted kernel H' = exp(beta K K^T - M): every
+    // entry is at most 1 (Cauchy-Schwarz), the diagonal's maximum is 1, and the
+    // pivots, the stop rule (relative to the diagonal's maximum) and the weights
+    // do not change; F is H's factor times exp(-M / 2).
+    double shift = 0.0;
+    if (alive) {
+        shift = __longlong_as_double((long long)__ldcg(&us->hmax_bits));
+        if (!isfinite(shift)) {
+            if (tid == 0) record_status(status, WC_ERR_NUMERIC);
+            alive = false;
+        }
+    }
+    for (int il = tid; il < mlen; il += kThreads) dg[il] = exp(dg[il] - shift);
     __syncthreads();  // the scan chunks below span rows that other threads initialised
-
     {
         int lo, hi;
         chunk_of(tid, mlen, &lo, &hi);
@@ -290,15 +303,8 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         const double tot = block_scan(sum, scan);
         if (tid == 0) part[blk] = tot;
     }
-    bool alive = unit_barrier(&us->bar, a.C, 1, a.timeout_ns, status, &bc.ok);
-    double hmax = 0.0;
-    if (alive) {
-        hmax = __longlong_as_double((long long)__ldcg(&us->hmax_bits));
-        if (!isfinite(hmax)) {
-            if (tid == 0) record_status(status, WC_ERR_NUMERIC);
-            alive = false;
-        }
-    }
+    if (alive) alive = unit_barrier(&us->bar, a.C, 2, a.timeout_ns, status, &bc.ok);
+    const double hmax = 1.0;  // the shifted diagonal's maximum
 
     int final_rank = alive ? r : 0;
     for (int j = 0; alive && j < r; ++j) {
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             for (int k = 0; k < kGroup; ++k) {
                 const int il = il0 + k;
                 double f = 0.0;
-                if (il < mlen && !ispiv[il]) f = (exp(a.beta * dot[k]) - cor[k]) / root;
+                if (il < mlen && !ispiv[il]) f = (exp(a.beta * dot[k] - shift) - cor[k]) / root;
                 out[k] = (float)f;
                 if (il < mlen) {
                     const double nd = dg[il] - f * f;
@@ -444,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             const double tot = block_scan(sum, scan);
             if (tid == 0) part[(size_t)((j + 1) & 1) * kMaxBlocksPerUnit + blk] = tot;
         }
-        if (!unit_barrier(&us->bar, a.C, (uint32_t)j + 2u, a.timeout_ns, status, &bc.ok)) {
+        if (!unit_barrier(&us->bar, a.C, (uint32_t)j + 3u, a.timeout_ns, status, &bc.ok)) {
             final_rank = j + 1;
             alive = false;
             break;

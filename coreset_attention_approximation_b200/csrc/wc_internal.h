@@ -24,7 +24,7 @@ struct UnitSync {
     int32_t s;                    // published pivot
     int32_t stop;                 // 1 when the run ends at the published step
     double d_s;                   // residual diagonal at the published pivot
-    unsigned long long hmax_bits; // max_i H_ii (bits of a positive double)
+    unsigned long long hmax_bits; // M = max_i beta |k_i|^2 (bits of a non-negative double)
     uint32_t pad[8];
 };
 static_assert(sizeof(UnitSync) == 64, "UnitSync is 64 bytes");
@@ -48,6 +48,7 @@ struct WsLayout {
     size_t kk;        // double[units]          |mean|^2
     size_t cdot;      // double[units][n]       <k_i, mean>
     size_t bias;      // float[units * bins][stride]  -beta log2(e) <k_i, mean> per bin, padded
+    size_t shift;     // double[units * bins]   M = max_i beta |k_i|^2 per bin unit (the factor's shift)
     size_t scratch_end;
     // room for outputs that wc_forward keeps in the workspace when not given
     size_t piv, rank, f, ks, w;
@@ -89,6 +90,9 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
 // the per-bin logit bias); `s` may be either view.
 wc_status launch_center(const Shape& s, const void* K, char* ws, cudaStream_t st);
 int center_bias_stride(const Shape& s);  // floats per bin row of the bias
+// M = max_i beta |k_i|^2 of every bin unit (centred keys when s.center), as the
+// selection computes it; the weights step divides the shift back out.
+wc_status launch_key_shift(const Shape& s, const void* K, char* ws, cudaStream_t st);
 wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const float* W,
                         const int32_t* rank, float* out, char* ws, cudaStream_t st);
 wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st);

@@ -40,19 +40,20 @@ __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict
 
 // C1 from the partial sums of the key splits, in fp64:
 //   C1[a, c] = e^(M + rho_a) sum_s e^{m_s - M} O_s[a, c],  M = max_s m_s
-// written column-major, Ct[u, c, a], for the solves.  rho_a = 0, or with
-// centred keys beta (|kbar|^2 - <k_s, kbar>) for the pivot s of row a (the
+// written column-major, Ct[u, c, a], for the solves.  rho_a = -shift_u (the
+// factor's shift, so that C1 is taken of the same shifted kernel as L), plus,
+// with centred keys, beta (|kbar|^2 - <k_s, kbar>) for the pivot s of row a (the
 // per-row factor of the centred kernel).  One block per (a, u).
 __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t* __restrict__ rank, double* Ct,
                                 int nsplit, int r, int dv, const int32_t* __restrict__ piv,
                                 const double* __restrict__ cdot, const double* __restrict__ kk, int bins, int n_all,
-                                double beta) {
+                                double beta, const double* __restrict__ shift) {
     const int a = blockIdx.x, u = blockIdx.y;
     if (a >= rank[u]) return;
-    double rho = 0.0;
+    double rho = -shift[u];
     if (cdot) {
         const int uc = u / bins;  // the caller's unit
-        rho = beta * (kk[uc] - cdot[(size_t)uc * n_all + piv[(size_t)u * r + a]]);
+        rho += beta * (kk[uc] - cdot[(size_t)uc * n_all + piv[(size_t)u * r + a]]);
     }
     const int w = c1_row(dv), wcols = dv + 1;
     const float* part = c1part + (size_t)u * nsplit * r * w;
@@ -284,7 +285,8 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
     merge_c1_kernel<<<dim3(s.r, s.units), 160, 0, st>>>(
         reinterpret_cast<const float*>(ws + L.c1part), rank, Ct, s.nsplit, s.r, s.dv, piv,
         s.center ? reinterpret_cast<const double*>(ws + L.cdot) : nullptr,
-        s.center ? reinterpret_cast<const double*>(ws + L.kk) : nullptr, s.bins, s.n_all, s.beta);
+        s.center ? reinterpret_cast<const double*>(ws + L.kk) : nullptr, s.bins, s.n_all, s.beta,
+        reinterpret_cast<const double*>(ws + L.shift));
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
     // as many right-hand sides per block as shared memory holds for this r
     const float* Lg = reinterpret_cast<const float*>(ws + L.lg);

@@ -36,7 +36,9 @@
  *                               entries >= rank are -1
  *       rank[B, Hkv]            int32, pivots accepted (<= r)
  *       F   [B, Hkv, r, ldf]    fp32, ldf = wc_f_ld(n_k); F[.., c, i] is the
- *                               factor entry of key i in column c; columns
+ *                               factor entry of key i in column c of the
+ *                               shifted kernel exp(beta K K^T - M_u), M_u =
+ *                               max_i beta |k_i|^2 (see select); columns
  *                               >= rank and entries i >= n_k are zero
  *       Ks  [B, Hkv, r, d]      dtype, the pivot keys K[piv]; rows >= rank zero
  *       W   [B, Hkv, r, dv+1]   fp32; rows >= rank zero
@@ -123,8 +125,12 @@ size_t wc_workspace_bytes(const wc_shape* shape);
 size_t wc_forward_workspace_bytes(const wc_shape* shape);
 
 /*
- * select — RPCholesky [Methodik item 1].  For each (b, kv head) unit u = b*Hkv+h:
- *   d_i = H_ii = exp(beta |k_i|^2);   for j = 0 .. r-1:
+ * select — RPCholesky [Methodik item 1].  For each (b, kv head) unit u = b*Hkv+h,
+ * on the kernel shifted in the log domain, H = exp(beta K K^T - M_u) with
+ * M_u = max_i beta |k_i|^2: every entry is then at most 1 (the factor cannot
+ * overflow), and the pivots, the stop rule and the weights are those of the
+ * unshifted kernel; F is the unshifted kernel's factor times exp(-M_u / 2).
+ *   d_i = H_ii = exp(beta |k_i|^2 - M_u);   for j = 0 .. r-1:
  *     u_j = Philox4x32-10(ctr = (j, u, 0, 0), key = seed).x0 * 2^-32
  *     s_j = smallest i with d_0 + ... + d_i > u_j * sum(d)  (inverse CDF)
  *     stop (rank = j) if sum(d) <= 0 or d_{s_j} <= eps_stop * max_i H_ii

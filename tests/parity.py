@@ -20,6 +20,15 @@ def rel_err(got, want) -> float:
     return float(np.max(np.abs(got - want)) / den) if den > 0 else float(np.max(np.abs(got)))
 
 
+def factor_shift(K, beta, center=False) -> float:
+    """M = max_i beta |k_i|^2 of one unit's (or bin's) keys: the library's F is
+    the factor of exp(beta K K^T - M), the oracle's F times exp(-M / 2)."""
+    Kd = np.asarray(K, dtype=np.float64)
+    if center:
+        Kd = Kd - Kd.mean(axis=0, keepdims=True)
+    return float(beta * np.max(np.sum(Kd * Kd, axis=1)))
+
+
 def run_gpu(Q, K, V, r, seed=0, **kw):
     dev = torch.device("cuda")
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
@@ -55,7 +64,8 @@ def compare(Q, K, V, r, seed=0, eps_stop=None, check_F=True, tol_w=None, **kw):
             assert np.array_equal(piv_g[b, h], o["piv"][b, h])
             if check_F:
                 Fg = g["F"][b, h].numpy()[:, :n].T          # n x r
-                report["err_F"] = max(report["err_F"], rel_err(Fg, o["F"][b, h]))
+                M = factor_shift(K[b, h].double().numpy(), o["beta"])
+                report["err_F"] = max(report["err_F"], rel_err(Fg, o["F"][b, h] * np.exp(-M / 2)))
                 assert np.all(g["F"][b, h].numpy()[:, n:] == 0.0)
             if k > 0:
                 report["err_W"] = max(report["err_W"], rel_err(g["W"][b, h].numpy()[:k], o["W"][b, h, :k]))
@@ -97,7 +107,11 @@ def compare_next(Q, K, V, r, seed=0, bins=1, center=False, check_F=True, tol_w=N
                 if check_F:
                     Fg = g["F"][b, h].numpy().reshape(nb, rb, -1)[bb][:, :nbk].T if nb > 1 else \
                         g["F"][b, h].numpy()[:, :n].T
-                    Fo = o["F"][b, h, bb * nbk:(bb + 1) * nbk, bb * rb:(bb + 1) * rb]
+                    Kc = K[b, h].double().numpy()
+                    if center:
+                        Kc = Kc - Kc.mean(axis=0, keepdims=True)
+                    M = factor_shift(Kc[bb * nbk:(bb + 1) * nbk], o["beta"])
+                    Fo = o["F"][b, h, bb * nbk:(bb + 1) * nbk, bb * rb:(bb + 1) * rb] * np.exp(-M / 2)
                     report["err_F"] = max(report["err_F"], rel_err(Fg, Fo))
                 rows = slice(bb * rb, bb * rb + k)
                 if k > 0:

@@ -144,9 +144,10 @@ def test_full_long_workload_prefix_and_properties():
         assert np.all(np.triu(L, 1) == 0.0) and np.all(np.diag(L) > 0.0)
         # F F^T reproduces H on sampled pivot rows
         Kh = K[0, h].double().numpy()
+        M = beta * np.max(np.sum(Kh * Kh, axis=1))   # F is the factor of exp(beta K K^T - M)
         for a in rng.choice(w.r, 4, replace=False):
             i = rng.choice(w.n_k, 64, replace=False)
-            Hrow = np.exp(beta * Kh[i] @ Kh[p[a]])
+            Hrow = np.exp(beta * Kh[i] @ Kh[p[a]] - M)
             FFt = F[0, h][:, i].double().numpy().T @ L[a].astype(np.float64)
             assert rel_err(FFt, Hrow) <= 1e-4
     # outputs of sampled queries of head 0 from the GPU's coreset and weights
@@ -180,3 +181,19 @@ def test_other_head_widths_bf16(d, dv):
     # (32, 96) runs on CUDA cores, the others on the tensor-core kernel
     w = WORKLOADS["vit"].replace(batch=1, hq=4, hkv=2, n_k=1500, n_q=300, d=d, dv=dv, r=100)
     compare(*make_inputs(w, seed=d + dv), w.r, seed=3)
+
+
+def test_large_key_norms_factor_stays_finite():
+    """Keys with beta |k|^2 around 300 (norms near 50 at d = 64): the unshifted
+    factor would reach exp(150) and overflow fp32; the selection works on the
+    kernel shifted by M = max beta |k_i|^2, so F stays finite and the pivots,
+    weights and outputs match the oracle's (fp64, unshifted)."""
+    w = WORKLOADS["vit"].replace(batch=1, hq=2, hkv=2, n_k=512, n_q=64, r=32)
+    Q, K, V = make_inputs(w, seed=21)
+    g = torch.Generator().manual_seed(21)
+    scale = 50.0 / K.double().norm(dim=-1, keepdim=True).clamp_min(1e-3)
+    K = (K.double() * scale * (0.8 + 0.2 * torch.rand(K.shape[:-1] + (1,), generator=g, dtype=torch.float64))).to(K.dtype)
+    Q = (Q.double() * 0.02).to(Q.dtype)
+    rep = compare(Q, K, V, w.r, seed=21, tol_w=2e-3)
+    res = run_gpu(Q, K, V, w.r, seed=21)
+    assert torch.isfinite(res["F"]).all() and res["F"].abs().max() <= 1.0 + 1e-6, rep
