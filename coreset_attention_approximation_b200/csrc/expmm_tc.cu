@@ -553,56 +553,52 @@ __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __
         dst[i] = __float2half_rn(__bfloat162float(src[i]));
 }
 
-// Weights for the attention GEMM: per unit and column c < dv, sigma_c =
-// max_s |W[s, c]| (1 if the column is zero), W16[s, c] = W[s, c] / sigma_c
-// (fp16) and wn[s] = W[s, dv], zero-padded to r_pad rows.  Rows >= the
-// unit's rank are zero (all r rows count with `all_keys`).
-// Column maxima: block (unit, 32 columns), 8 row groups of 32 threads.
-__global__ void weights_sigma_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, float* sigma,
-                                     int r, int dv, int all_keys) {
-    const int u = blockIdx.x, c = blockIdx.y * 32 + (threadIdx.x & 31), g = threadIdx.x >> 5;
+// The attention's weights as the tensor cores take them: per unit and value
+// column c, sigma_c = max_s |W[s][c]| over the live rows (1 for an all-zero
+// column), W16[s][c] = fp16(W[s][c] / sigma_c) (zero rows up to r), and the
+// normaliser column wn[s] = W[s][dv] in fp32 (zero up to r_pad).  One block per
+// (unit, 32 columns): warp g walks rows g, g + 32, ... so the row loop is 32
+// times shorter than the rank, then the block's maximum scales the same
+// columns it just read (from L2).
+constexpr int kPrepThreads = 1024;
+
+__global__ void __launch_bounds__(kPrepThreads) weights_prep_kernel(const float* __restrict__ W,
+                                                                    const int32_t* __restrict__ rank, float* sigma,
+                                                                    __half* W16, float* wn, int r, int r_pad, int dv,
+                                                                    int all_keys) {
+    constexpr int kWarps = kPrepThreads / 32;
+    const int u = blockIdx.x, lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+    const int c = blockIdx.y * 32 + lane;
     const int k = all_keys ? r : rank[u];
     const float* Wu = W + (size_t)u * r * (dv + 1);
     float mx = 0.f;
-    if (c < dv)
-        for (int s = g; s < k; s += 8) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
-    __shared__ float part[8][32];
-    part[g][threadIdx.x & 31] = mx;
+    if (c < dv) {
+#pragma unroll 8
+        for (int s = g; s < k; s += kWarps) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
+    }
+    __shared__ float part[kWarps][33];
+    part[g][lane] = mx;
     __syncthreads();
-    if (g == 0 && c < dv) {
-        float m = part[0][threadIdx.x];
+    float m = 0.f;
 #pragma unroll
-        for (int i = 1; i < 8; ++i) m = fmaxf(m, part[i][threadIdx.x]);
-        sigma[(size_t)u * dv + c] = m > 0.f ? m : 1.f;
+    for (int i = 0; i < kWarps; ++i) m = fmaxf(m, part[i][lane]);
+    const float sg = m > 0.f ? m : 1.f;
+    if (c < dv) {
+        if (g == 0) sigma[(size_t)u * dv + c] = sg;
+        __half* Wh = W16 + (size_t)u * r * dv;
+#pragma unroll 4
+        for (int s = g; s < r; s += kWarps)
+            Wh[(size_t)s * dv + c] = __float2half_rn(s < k ? Wu[(size_t)s * (dv + 1) + c] / sg : 0.f);
     }
-}
-
-// The scaled fp16 weights and the normaliser column, grid-stride over every unit.
-__global__ void weights_half_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank,
-                                    const float* __restrict__ sigma, __half* W16, float* wn, int units, int r,
-                                    int r_pad, int dv, int all_keys) {
-    const size_t per = (size_t)r * dv, total = (size_t)units * per;
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-        const int u = (int)(e / per);
-        const int rem = (int)(e - (size_t)u * per);
-        const int s = rem / dv, c = rem - s * dv;
-        const int k = all_keys ? r : rank[u];
-        const float v = s < k ? W[((size_t)u * r + s) * (dv + 1) + c] / sigma[(size_t)u * dv + c] : 0.f;
-        W16[e] = __float2half_rn(v);
-    }
-    const size_t tw = (size_t)units * r_pad;
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < tw; e += (size_t)gridDim.x * blockDim.x) {
-        const int u = (int)(e / r_pad), s = (int)(e - (size_t)u * r_pad);
-        const int k = all_keys ? r : rank[u];
-        wn[e] = s < k ? W[((size_t)u * r + s) * (dv + 1) + dv] : 0.f;
-    }
+    if (blockIdx.y == 0)
+        for (int s = threadIdx.x; s < r_pad; s += kPrepThreads)
+            wn[(size_t)u * r_pad + s] = s < k ? Wu[(size_t)s * (dv + 1) + dv] : 0.f;
 }
 
 wc_status launch_weights_prep(const Shape& s, const float* W, const int32_t* rank, __half* W16, float* sigma,
                               float* wn, cudaStream_t st) {
-    weights_sigma_kernel<<<dim3(s.units, (s.dv + 31) / 32), 256, 0, st>>>(W, rank, sigma, s.r, s.dv, s.bins > 1);
-    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
-    weights_half_kernel<<<1184, 256, 0, st>>>(W, rank, sigma, W16, wn, s.units, s.r, s.r_pad, s.dv, s.bins > 1);
+    weights_prep_kernel<<<dim3(s.units, (s.dv + 31) / 32), kPrepThreads, 0, st>>>(W, rank, sigma, W16, wn, s.r,
+                                                                                 s.r_pad, s.dv, s.bins > 1);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 

@@ -196,8 +196,9 @@ def forward(Q, K, V, r, seed=0, *, ws=None, stream=None, outputs=None, **kw):
     """
     shape = shape_of(Q, K, V, r, seed=seed, **kw)
     o = dict(outputs or {})
-    for k, v in _outputs(shape, K.device, K.dtype).items():
-        o.setdefault(k, v)
+    if any(k not in o for k in ("piv", "rank", "F", "Ks", "W")):
+        for k, v in _outputs(shape, K.device, K.dtype).items():
+            o.setdefault(k, v)
     o.setdefault("out", torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], shape.dv, dtype=torch.float32,
                                     device=K.device))
     ws = workspace(shape, K.device) if ws is None else ws
@@ -219,6 +220,77 @@ def forward_host(Q, K, V, r, seed=0, *, device="cuda", ws=None, stream=None, **k
     out.copy_(res["out"], non_blocking=True)
     torch.cuda.current_stream().synchronize()
     return out
+
+
+class HostPipeline:
+    """Forward passes over a sequence of host batches, with the copies
+    overlapped: batch i+1's host-to-device copy and batch i-1's device-to-host
+    copy run on their own streams while batch i computes.  Two device copies
+    of Q, K, V and out alternate; the factor, weights and workspace are shared
+    (the passes themselves run one after another on the compute stream).
+
+    Host tensors must be pinned for the copies to overlap.  Every batch has
+    the shapes and dtype of the (Q, K, V) given here."""
+
+    def __init__(self, Q, K, V, r, seed=0, *, device="cuda", stream=None, ws=None, outputs=None, **kw):
+        """Q, K, V: host tensors of the batches' shapes and dtype (only their
+        shapes are read).  ws / outputs: optional workspace and (piv, rank, F,
+        Ks, W) device tensors to reuse; the last batch's stay there."""
+        self.device = torch.device(device)
+        self.r, self.seed, self.kw = r, seed, kw
+        self.shape = shape_of(Q, K, V, r, seed=seed, **kw)
+        self.ws = workspace(self.shape, self.device) if ws is None else ws
+        self.shared = {k: v for k, v in (outputs or {}).items() if k != "out"}
+        if any(k not in self.shared for k in ("piv", "rank", "F", "Ks", "W")):
+            for k, v in _outputs(self.shape, self.device, K.dtype).items():
+                self.shared.setdefault(k, v)
+        out_shape = (Q.shape[0], Q.shape[1], Q.shape[2], self.shape.dv)
+        self.bufs = [dict(Q=torch.empty(Q.shape, dtype=Q.dtype, device=self.device),
+                          K=torch.empty(K.shape, dtype=K.dtype, device=self.device),
+                          V=torch.empty(V.shape, dtype=V.dtype, device=self.device),
+                          out=torch.empty(out_shape, dtype=torch.float32, device=self.device)) for _ in range(2)]
+        self.compute = stream or torch.cuda.current_stream(self.device)
+        self.h2d = torch.cuda.Stream(self.device)
+        self.d2h = torch.cuda.Stream(self.device)
+        self.loaded = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.drained = [torch.cuda.Event() for _ in range(2)]
+        self.started = [False, False]
+
+    def run(self, batches):
+        """batches: iterable of (Q, K, V, out) host tensors; out [B, Hq, nq, dv]
+        fp32 receives the batch's output.  The copies and passes are queued
+        behind whatever the compute stream already holds; returns once the
+        last output has been queued (call `wait()` before reading it)."""
+        for i, (Qh, Kh, Vh, oh) in enumerate(batches):
+            j = i % 2
+            b = self.bufs[j]
+            with torch.cuda.stream(self.h2d):
+                if i == 0:
+                    self.h2d.wait_stream(self.compute)            # after whatever the caller queued
+                if self.started[j]:
+                    self.h2d.wait_event(self.computed[j])     # batch i-2 has finished reading buffer j
+                b["Q"].copy_(Qh, non_blocking=True)
+                b["K"].copy_(Kh, non_blocking=True)
+                b["V"].copy_(Vh, non_blocking=True)
+                self.loaded[j].record(self.h2d)
+            self.compute.wait_event(self.loaded[j])
+            if self.started[j]:
+                self.compute.wait_event(self.drained[j])       # batch i-2's output has left buffer j
+            forward(b["Q"], b["K"], b["V"], self.r, self.seed, ws=self.ws, stream=self.compute,
+                    outputs=dict(self.shared, out=b["out"]), **self.kw)
+            self.computed[j].record(self.compute)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(self.computed[j])
+                oh.copy_(b["out"], non_blocking=True)
+                self.drained[j].record(self.d2h)
+            self.started[j] = True
+        # the compute stream ends after the last copy out
+        self.compute.wait_stream(self.d2h)
+
+    def wait(self):
+        self.compute.synchronize()
+        return check_device_status(self.ws, self.compute)
 
 
 def check_device_status(ws, stream=None) -> int:

@@ -38,6 +38,16 @@ def test_kv_reduced_gqa():
     compare(*make_inputs(w), w.r, seed=3, tol_w=2e-3)
 
 
+def test_kv_full_workload_two_units():
+    """The KV-cache workload at full size (32 query heads over 8 kv heads,
+    n = 32768, r = 1024, 256 queries) in the bench's launch configuration: the
+    GPU runs all 8 units; the oracle checks every pivot, the factor, the weights
+    and the outputs of the first and last unit (8 query heads)."""
+    w = WORKLOADS["kv"]
+    rep = compare(*make_inputs(w), w.r, seed=0, tol_w=2e-3, units=[0, w.hkv - 1])
+    assert rep["err_out"] <= TOL_OUT[torch.bfloat16]
+
+
 def test_long_reduced_many_blocks_per_unit():
     w = WORKLOADS["long"].replace(hq=1, hkv=1, n_k=16384, n_q=2048, r=512)
     compare(*make_inputs(w), w.r, seed=5, tol_w=2e-3)
@@ -197,3 +207,23 @@ def test_large_key_norms_factor_stays_finite():
     rep = compare(Q, K, V, w.r, seed=21, tol_w=2e-3)
     res = run_gpu(Q, K, V, w.r, seed=21)
     assert torch.isfinite(res["F"]).all() and res["F"].abs().max() <= 1.0 + 1e-6, rep
+
+
+@pytest.mark.parametrize("bins", [1, 4])
+def test_host_pipeline_matches_forward(bins):
+    """Three different host batches through the double-buffered host pipeline
+    give, bit for bit, the outputs of separate forward calls (same seed)."""
+    w = WORKLOADS["diffusion"].replace(batch=1, hq=4, hkv=2, n_k=4096, n_q=1000, r=256)
+    batches = [make_inputs(w, seed=s) for s in (11, 12, 13)]
+    pinned = [tuple(t.pin_memory() for t in b) for b in batches]
+    outs = [torch.empty(w.batch, w.hq, w.n_q, w.dv, dtype=torch.float32).pin_memory() for _ in batches]
+    pipe = wildcat.HostPipeline(*pinned[0], w.r, seed=4, bins=bins)
+    pipe.run([(q, k, v, o) for (q, k, v), o in zip(pinned, outs)])
+    assert pipe.wait() == 0
+    for (Q, K, V), o in zip(batches, outs):
+        ref = run_gpu(Q, K, V, w.r, seed=4, bins=bins)["out"]
+        assert torch.equal(o, ref)
+    # a second run on the same pipeline (buffers and events reused)
+    pipe.run([(*pinned[2], outs[0])])
+    assert pipe.wait() == 0
+    assert torch.equal(outs[0], outs[2])
