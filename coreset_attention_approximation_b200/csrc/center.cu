@@ -98,34 +98,50 @@ wc_status launch_center_t(const Shape& s, const void* K, char* ws, cudaStream_t 
 }
 
 // M[u'] = max over bin unit u''s keys of beta |k_i|^2 (k_i - kbar when centred),
-// each |.|^2 summed in fp64 in dimension order as the selection sums it, so
-// the two agree bit for bit.  Blocks (chunk of kShiftChunk keys, bin unit);
-// the block maxima meet in an atomic maximum on the bits (non-negative doubles
-// order like their bits; a maximum is exact, so the result is deterministic).
-constexpr int kShiftChunk = 2048;
+// in fp64.  A warp takes kShiftKeys keys at a time, lane l summing dimensions
+// l, l + 32, ... of each (coalesced loads, all of them issued before the sums
+// when the head width DT is a compile-time constant), then a fixed shuffle tree
+// adds the lanes, so the result is deterministic; it may differ from the
+// selection's own sum in the last bits, which scales W by 1 + O(1e-16 M) (the
+// row normalisation cancels it).  The warp maxima meet in an atomic maximum on
+// the bits (non-negative doubles order like their bits; a maximum is exact).
+constexpr int kShiftBlocks = 2048;  // about two waves of 256-thread blocks on 148 SMs
+constexpr int kShiftKeys = 4;
 
-template <typename T>
+template <typename T, int DT>
 __global__ void key_shift_kernel(const T* __restrict__ K, const double* __restrict__ kbar,
-                                 unsigned long long* shift_bits, int n, int d, int bins, double beta) {
+                                 unsigned long long* shift_bits, int n, int d_rt, int bins, double beta) {
+    const int d = DT ? DT : d_rt;
     const int ub = blockIdx.y;               // bin unit: caller unit ub / bins, bin ub % bins
     const int nb = n / bins;
     const T* Kb = K + (size_t)ub * nb * d;   // the bin's keys are contiguous
     const double* m = kbar ? kbar + (size_t)(ub / bins) * d : nullptr;
-    const int i0 = blockIdx.x * kShiftChunk, i1 = min(nb, i0 + kShiftChunk);
+    const int lane = threadIdx.x & 31, warps = blockDim.x >> 5;
+    const int gw = blockIdx.x * warps + (int)(threadIdx.x >> 5), nw = gridDim.x * warps;
     double mx = 0.0;
-    for (int i = i0 + (int)threadIdx.x; i < i1; i += blockDim.x) {
-        const T* k = Kb + (size_t)i * d;
-        double ss = 0.0;
-        for (int c = 0; c < d; ++c) {
-            double x = (double)to_f32(k[c]);
-            if (m) x -= m[c];
-            ss += x * x;
-        }
-        mx = fmax(mx, beta * ss);
-    }
+    for (int i0 = gw * kShiftKeys; i0 < nb; i0 += nw * kShiftKeys) {
+        double ss[kShiftKeys];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((threadIdx.x & 31) == 0 && mx > 0.0) atomicMax(shift_bits + ub, (unsigned long long)__double_as_longlong(mx));
+        for (int q = 0; q < kShiftKeys; ++q) {
+            ss[q] = 0.0;
+            if (i0 + q < nb) {
+                const T* k = Kb + (size_t)(i0 + q) * d;
+#pragma unroll
+                for (int c = lane; c < d; c += 32) {
+                    double x = (double)to_f32(k[c]);
+                    if (m) x -= m[c];
+                    ss[q] += x * x;
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kShiftKeys; ++q) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], o);
+            mx = fmax(mx, beta * ss[q]);
+        }
+    }
+    if (lane == 0 && mx > 0.0) atomicMax(shift_bits + ub, (unsigned long long)__double_as_longlong(mx));
 }
 
 template <typename T>
@@ -134,9 +150,16 @@ wc_status launch_key_shift_t(const Shape& s, const void* K, char* ws, cudaStream
     const double* kbar = s.center ? reinterpret_cast<const double*>(ws + L.kbar) : nullptr;
     const int ub = s.units_all * s.bins, nb = s.n_all / s.bins;
     if (cudaMemsetAsync(ws + L.shift, 0, sizeof(double) * ub, st) != cudaSuccess) return WC_ERR_CUDA;
-    key_shift_kernel<T><<<dim3((nb + kShiftChunk - 1) / kShiftChunk, ub), 256, 0, st>>>(
-        static_cast<const T*>(K), kbar, reinterpret_cast<unsigned long long*>(ws + L.shift), s.n_all, s.d, s.bins,
-        s.beta);
+    const int per_bin = (kShiftBlocks + ub - 1) / ub, need = (nb + 8 * kShiftKeys - 1) / (8 * kShiftKeys);
+    const dim3 grid(per_bin < need ? per_bin : need, ub);
+    const T* Kt = static_cast<const T*>(K);
+    auto* bits = reinterpret_cast<unsigned long long*>(ws + L.shift);
+    if (s.d == 128)
+        key_shift_kernel<T, 128><<<grid, 256, 0, st>>>(Kt, kbar, bits, s.n_all, s.d, s.bins, s.beta);
+    else if (s.d == 64)
+        key_shift_kernel<T, 64><<<grid, 256, 0, st>>>(Kt, kbar, bits, s.n_all, s.d, s.bins, s.beta);
+    else
+        key_shift_kernel<T, 0><<<grid, 256, 0, st>>>(Kt, kbar, bits, s.n_all, s.d, s.bins, s.beta);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
