@@ -362,18 +362,11 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "copies": "double-buffered: step i+1 in and step i-1 out overlap step i"},
-        "gpu_launches": (LAUNCHES_PER_STEP + (CENTER_LAUNCHES if args.center else 0)) * args.steps,
+        # counted on the profiled step (the same launches as every timed step)
+        "gpu_launches": kernels.pop("launches") * args.steps,
         "clocks": clocks.summary(),
     }
     return res
-
-
-# select (1 cooperative wave here), the factor's shift for the weights, gather, fp16
-# copy of V, C1 exp-GEMM, merge of the C1 partials, triangular solves, fp16
-# weights with their column scales, attention exp-GEMM
-LAUNCHES_PER_STEP = 9
-# centring: column sums, mean, key-mean dots, once in the select and once in the weights
-CENTER_LAUNCHES = 6
 
 
 def kernel_breakdown(step):
@@ -387,19 +380,23 @@ def kernel_breakdown(step):
         torch.cuda.synchronize()
     import re
 
-    out = {}
+    out = {"launches": 0}
     for ev in prof.events():
         if ev.device_type.name != "CUDA":
             continue
         name = ev.name
+        if "wc::" in name:
+            out["launches"] += 1          # this library's kernels (namespace wc)
         short = None
         m = re.search(r"expmm_(tc|simt)_kernel<[^>]*?(\d)>", name)
         if m:
-            short = "attend_gemm" if m.group(2) == "1" else "weights_gemm"  # modes 0, 2: weights; 1: attention
+            # modes 0, 2: the weights' partial sums; 1: attention; 3: attention over a key split
+            short = "attend_gemm" if m.group(2) in ("1", "3") else "weights_gemm"
         else:
             for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
                              ("merge_c1", "merge_c1"), ("trsm_kernel", "solve"),
-                             ("weights_prep", "w_prep"), ("key_shift", "shift")):
+                             ("weights_prep", "w_prep"), ("key_shift", "shift"),
+                             ("attend_combine", "attend_combine")):
                 if key in name:
                     short = tag
                     break

@@ -99,6 +99,7 @@ WsLayout make_layout(const Shape& s) {
     L.cdot = take(C * sizeof(double) * U * n);
     L.bias = take(C * sizeof(float) * U * B * ((nb + 127) / 128 * 128));
     L.shift = take(sizeof(double) * U * B);
+    L.apart = take(sizeof(float) * attend_split_floats(s));
     L.scratch_end = off;
     L.piv = take(sizeof(int32_t) * U * r);
     L.rank = take(sizeof(int32_t) * U * B);

@@ -25,6 +25,7 @@
 // swizzled canonical layouts: A, B and P K-major, C MN-major.  Every wait is
 // bounded; a wait that runs out records WC_ERR_TIMEOUT and the block winds
 // down (drains its copies and MMAs, frees TMEM) instead of hanging.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -76,10 +77,13 @@ struct TcArgs {
     int bias_stride;
 };
 
-// MODE: kExpmmPartial, kExpmmRownorm, or kModeBias = partial sums of
+// MODE: kExpmmPartial, kExpmmRownorm, kModeBias = partial sums of
 // exp(beta <a, b_j> + bias_j) (the centred kernel: the bias tile arrives with
-// the value tile).
+// the value tile), or kModeAttnSplit = attention over one split of the
+// coreset (blockIdx.y), written as an unnormalised partial row (O scaled by the
+// column scales | normaliser share | reference) for attend_combine_kernel.
 constexpr int kModeBias = 2;
+constexpr int kModeAttnSplit = 3;
 
 template <int D, int DV>
 struct Smem {
@@ -106,6 +110,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     expmm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                     const __grid_constant__ CUtensorMap mapC, const TcArgs args) {
     using L = Smem<D, DV>;
+    // A holds queries (rows mapped to kv units by the query-head group), the
+    // normaliser is weighted by the coreset's normaliser column, and the value
+    // columns carry scales; only kExpmmRownorm divides the rows out in place
+    constexpr bool kQueries = MODE == kExpmmRownorm || MODE == kModeAttnSplit;
+    constexpr bool kNormOut = MODE == kExpmmRownorm;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = smem_raw;
     if (smem_u32(sm) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -128,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int z = blockIdx.z;
     int unit, a_valid, b_lo, b_hi, split = 0, a_row0;
-    if (MODE != kExpmmRownorm) {
+    if (!kQueries) {
         unit = z;
         a_valid = args.rank[unit];
         split = blockIdx.y;
@@ -139,8 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hkv = args.hq / args.group;
         unit = (z / args.hq) * hkv + (z % args.hq) / args.group;
         a_valid = args.a_rows;
-        b_lo = 0;
-        b_hi = args.all_keys ? args.b_rows : args.rank[unit];
+        const int b_all = args.all_keys ? args.b_rows : args.rank[unit];
+        split = MODE == kModeAttnSplit ? (int)blockIdx.y : 0;
+        b_lo = split * args.split_len;
+        b_hi = min(b_all, b_lo + args.split_len);
         a_row0 = z * args.a_head_rows + blockIdx.x * BM;
     }
     const int a0 = blockIdx.x * BM;
@@ -210,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         unsigned char* st = sm + L::C0 + s * L::kC;
     #pragma unroll
                         for (int c = 0; c < DV / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapC, &fl[s], c * 64, brow);
-                        if (MODE == kExpmmRownorm)
+                        if (kQueries)
                             bulk_load(sm + L::Wv + s * BN * 4, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN,
                                       BN * 4, &fl[s]);
                         if (MODE == kModeBias)
@@ -366,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mO = mn;
             }
             if (t + 1 < T) tok[row] = mn;       // the partner reads it after this tile's hand-over below
-            if (ok && MODE == kExpmmRownorm) {
+            if (ok && kQueries) {
                 // w arrives with the value tile; this stage cannot be reloaded before PV(t)
                 ok = mbar_wait(&fullC[t % NC], (t / NC) & 1, abort_flag, args.status, kTcTimeoutNs);
                 ok = __all_sync(0xffffffffu, ok);
@@ -387,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const float* sh = sv + 32 * h;
                     uint32_t packed[16];
-                    float w[MODE == kExpmmRownorm ? 32 : 1];
-                    if (MODE == kExpmmRownorm) {
+                    float w[kQueries ? 32 : 1];
+                    if (kQueries) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
                             const float4 f = lds_f4_ordered(wv + 32 * h + j);
@@ -408,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             p0 = ex2_ordered(fmaf(sh[j], cb, nm));
                             p1 = ex2_ordered(fmaf(sh[j + 1], cb, nm));
                         }
-                        if (MODE == kExpmmRownorm)
+                        if (kQueries)
                             lp[(j >> 1) & 3] = fmaf(p1, w[j + 1], fmaf(p0, w[j], lp[(j >> 1) & 3]));
                         else
                             lp[(j >> 1) & 3] += p0 + p1;
@@ -455,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // share of the normaliser in its own reference; the last one adds the
         // two in the final reference and hands the total back.
         // the column scales of the attention output, loaded before the waits below
-        float sgv[MODE == kExpmmRownorm ? DV / 2 : 1];
-        if (MODE == kExpmmRownorm) {
+        float sgv[kQueries ? DV / 2 : 1];
+        if (kQueries) {
             const float4* s4 = reinterpret_cast<const float4*>(args.sigma + (size_t)unit * DV + par * (DV / 2));
 #pragma unroll
             for (int c = 0; c < DV / 2; c += 4) {
@@ -498,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* stg = reinterpret_cast<float*>(sm + L::C0);
         const bool have_o = ok && T > 0;
         const uint32_t tO = tO0 + lanes + par * (DV / 2);
-        const float inv = 1.f / lt;
+        const float inv = kNormOut ? 1.f / lt : 1.f;
         float* srow = stg + row * SST + par * (DV / 2);
 #pragma unroll
         for (int c0 = 0; c0 < DV / 2; c0 += 32) {
@@ -513,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
                 float4 v = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-                if (MODE == kExpmmRownorm) {
+                if (kQueries) {
                     v.x *= sgv[c0 + c] * inv;
                     v.y *= sgv[c0 + c + 1] * inv;
                     v.z *= sgv[c0 + c + 2] * inv;
@@ -522,18 +533,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<float4*>(srow + c0 + c) = v;
             }
         }
-        if (MODE != kExpmmRownorm && last) *reinterpret_cast<float2*>(stg + row * SST + DV) = make_float2(lt, mO * kLn2);
+        if (!kNormOut && last) *reinterpret_cast<float2*>(stg + row * SST + DV) = make_float2(lt, mO * kLn2);
         fence_async_smem();                     // the bulk copies read the staged rows through the async proxy
         softmax_sync();                         // all 8 softmax warps have staged their part
         const int rows = min(BM, a_valid - a0);
         const int st = tid - 4 * 32;            // 0 .. 255
-        if (ok && MODE != kExpmmRownorm && st == 0) {
-            bulk_store(static_cast<float*>(args.out) + (((size_t)unit * args.nsplit + split) * args.r + a0) * SST, stg,
-                       (uint32_t)(rows * SST * 4));
+        if (ok && !kNormOut && st == 0) {
+            const size_t prow = kQueries ? ((size_t)z * args.nsplit + split) * args.a_rows + a0
+                                         : ((size_t)unit * args.nsplit + split) * args.r + a0;
+            bulk_store(static_cast<float*>(args.out) + prow * SST, stg, (uint32_t)(rows * SST * 4));
             bulk_commit();
             bulk_wait_read_all();
         }
-        if (ok && MODE == kExpmmRownorm && st < rows) {
+        if (ok && kNormOut && st < rows) {
             bulk_store(static_cast<float*>(args.out) + ((size_t)z * args.a_rows + a0 + st) * DV, stg + st * SST,
                        (uint32_t)(DV * 4));
             bulk_commit();
@@ -547,6 +559,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 2) tmem_dealloc<512>(tmem);
 }
 
+// Key-split attention: row q of query head h from its splits' partial rows
+// (O_s | l_s | m_s, m in natural-log units):
+//   out[h][q][c] = sum_s e_s O_s[c] / sum_s e_s l_s,  e_s = exp(m_s - max_s m_s).
+// One warp per query row, lanes over the value columns.
+template <int DV>
+__global__ void attend_combine_kernel(const float* __restrict__ part, float* __restrict__ out, int nq, int nsplit,
+                                      int rows_total) {
+    constexpr int SST = c1_row(DV);
+    const int wrow = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (wrow >= rows_total) return;
+    const int h = wrow / nq, qr = wrow - h * nq;
+    const size_t sstride = (size_t)nq * SST;                 // between splits
+    const float* p = part + ((size_t)h * nsplit * nq + qr) * SST;
+    float mx = -INFINITY;
+    for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, p[sp * sstride + DV + 1]);
+    float acc[DV / 32], lsum = 0.f;
+#pragma unroll
+    for (int k = 0; k < DV / 32; ++k) acc[k] = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) {
+        const float* ps = p + sp * sstride;
+        const float m = ps[DV + 1];
+        const float e = m == -INFINITY ? 0.f : expf(m - mx);
+        lsum = fmaf(e, ps[DV], lsum);
+#pragma unroll
+        for (int k = 0; k < DV / 32; ++k) acc[k] = fmaf(e, ps[lane + 32 * k], acc[k]);
+    }
+    const float inv = 1.f / lsum;
+    float* o = out + (size_t)wrow * DV;
+#pragma unroll
+    for (int k = 0; k < DV / 32; ++k) o[lane + 32 * k] = acc[k] * inv;
+}
+
 // V (bf16) -> fp16 copy for the value operand of the weights GEMM.
 __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, size_t count) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
@@ -556,49 +600,62 @@ __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __
 // The attention's weights as the tensor cores take them: per unit and value
 // column c, sigma_c = max_s |W[s][c]| over the live rows (1 for an all-zero
 // column), W16[s][c] = fp16(W[s][c] / sigma_c) (zero rows up to r), and the
-// normaliser column wn[s] = W[s][dv] in fp32 (zero up to r_pad).  One block per
-// (unit, 32 columns): warp g walks rows g, g + 32, ... so the row loop is 32
-// times shorter than the rank, then the block's maximum scales the same
-// columns it just read (from L2).
-constexpr int kPrepThreads = 1024;
+// normaliser column wn[s] = W[s][dv] in fp32 (zero up to r_pad).  A cluster of
+// kPrepCluster blocks per (unit, 32 columns); block q of the cluster takes rows
+// 8 q + g + 64 k (warp g), so every block walks r / 64 rows.  The blocks'
+// column maxima meet through distributed shared memory, then each block scales
+// the rows it just read (from L2).
+constexpr int kPrepCluster = 8;
+constexpr int kPrepWarps = 8;
 
-__global__ void __launch_bounds__(kPrepThreads) weights_prep_kernel(const float* __restrict__ W,
-                                                                    const int32_t* __restrict__ rank, float* sigma,
-                                                                    __half* W16, float* wn, int r, int r_pad, int dv,
-                                                                    int all_keys) {
-    constexpr int kWarps = kPrepThreads / 32;
-    const int u = blockIdx.x, lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+__global__ void __cluster_dims__(kPrepCluster, 1, 1) __launch_bounds__(kPrepWarps * 32)
+    weights_prep_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, float* sigma, __half* W16,
+                        float* wn, int r, int r_pad, int dv, int all_keys) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int q = (int)cluster.block_rank();
+    const int u = blockIdx.x / kPrepCluster, lane = threadIdx.x & 31, g = threadIdx.x >> 5;
     const int c = blockIdx.y * 32 + lane;
     const int k = all_keys ? r : rank[u];
     const float* Wu = W + (size_t)u * r * (dv + 1);
+    const int s0 = q * kPrepWarps + g, step = kPrepCluster * kPrepWarps;
     float mx = 0.f;
     if (c < dv) {
-#pragma unroll 8
-        for (int s = g; s < k; s += kWarps) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
+#pragma unroll 4
+        for (int s = s0; s < k; s += step) mx = fmaxf(mx, fabsf(Wu[(size_t)s * (dv + 1) + c]));
     }
-    __shared__ float part[kWarps][33];
+    __shared__ float part[kPrepWarps][33];
+    __shared__ float bmax[32];
     part[g][lane] = mx;
     __syncthreads();
+    if (g == 0) {
+        float m = part[0][lane];
+#pragma unroll
+        for (int i = 1; i < kPrepWarps; ++i) m = fmaxf(m, part[i][lane]);
+        bmax[lane] = m;
+    }
+    cluster.sync();                            // every block's maxima are in its shared memory
     float m = 0.f;
 #pragma unroll
-    for (int i = 0; i < kWarps; ++i) m = fmaxf(m, part[i][lane]);
+    for (int p = 0; p < kPrepCluster; ++p) m = fmaxf(m, cluster.map_shared_rank(bmax, p)[lane]);
+    cluster.sync();                            // no block leaves while a peer still reads its maxima
     const float sg = m > 0.f ? m : 1.f;
     if (c < dv) {
-        if (g == 0) sigma[(size_t)u * dv + c] = sg;
+        if (q == 0 && g == 0) sigma[(size_t)u * dv + c] = sg;
         __half* Wh = W16 + (size_t)u * r * dv;
 #pragma unroll 4
-        for (int s = g; s < r; s += kWarps)
+        for (int s = s0; s < r; s += step)
             Wh[(size_t)s * dv + c] = __float2half_rn(s < k ? Wu[(size_t)s * (dv + 1) + c] / sg : 0.f);
     }
     if (blockIdx.y == 0)
-        for (int s = threadIdx.x; s < r_pad; s += kPrepThreads)
+        for (int s = q * kPrepWarps * 32 + (int)threadIdx.x; s < r_pad; s += step * 32)
             wn[(size_t)u * r_pad + s] = s < k ? Wu[(size_t)s * (dv + 1) + dv] : 0.f;
 }
 
 wc_status launch_weights_prep(const Shape& s, const float* W, const int32_t* rank, __half* W16, float* sigma,
                               float* wn, cudaStream_t st) {
-    weights_prep_kernel<<<dim3(s.units, (s.dv + 31) / 32), kPrepThreads, 0, st>>>(W, rank, sigma, W16, wn, s.r,
-                                                                                 s.r_pad, s.dv, s.bins > 1);
+    weights_prep_kernel<<<dim3(s.units * kPrepCluster, (s.dv + 31) / 32), kPrepWarps * 32, 0, st>>>(
+        W, rank, sigma, W16, wn, s.r, s.r_pad, s.dv, s.bins > 1);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -654,6 +711,26 @@ wc_status launch_tc(int d, int dv, const CUtensorMap& A, const CUtensorMap& B, c
 }
 
 }  // namespace
+
+int attend_splits(const Shape& s) {
+    // the attention's query tiles alone fill the GPU: no split
+    if (s.dtype != WC_BF16 || !((s.d == 64 || s.d == 128) && (s.dv == 64 || s.dv == 128))) return 1;
+    const long base = (long)((s.nq + BM - 1) / BM) * s.batch * s.hq;
+    const int tiles = (s.r + BN - 1) / BN;
+    if (base == 0 || tiles < 2) return 1;
+    // as many splits as keep every block in one wave (one block per SM): a
+    // second wave would cost a whole block's fixed prologue and epilogue again
+    int want = (int)(kAttendFill / base);
+    if (want < 2) return 1;
+    if (want > tiles) want = tiles;
+    const int per = (tiles + want - 1) / want;               // key tiles per split
+    return (tiles + per - 1) / per;
+}
+
+size_t attend_split_floats(const Shape& s) {
+    const int ns = attend_splits(s);
+    return ns > 1 ? (size_t)s.batch * s.hq * ns * s.nq * c1_row(s.dv) : 0;
+}
 
 bool tc_supported(const Shape& s) {
     return s.dtype == WC_BF16 && (s.d == 64 || s.d == 128) && (s.dv == 64 || s.dv == 128) && encode_fn() != nullptr;
@@ -723,8 +800,27 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     a.group = s.hq / s.hkv;
     a.all_keys = s.bins > 1;
     a.cb = (float)(s.beta * 1.4426950408889634);
-    dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
-    return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
+    const int ns = attend_splits(s);
+    if (ns <= 1) {
+        dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
+        return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
+    }
+    // few query tiles: split the coreset over blockIdx.y, then combine the partial rows
+    const int tiles = (s.r + BN - 1) / BN;
+    float* part = reinterpret_cast<float*>(ws + Lw.apart);
+    a.out = part;
+    a.nsplit = ns;
+    a.split_len = (tiles + ns - 1) / ns * BN;
+    dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), ns, s.batch * s.hq);
+    wc_status e = launch_tc<kModeAttnSplit>(s.d, s.dv, mA, mB, mC, a, grid, st);
+    if (e != WC_OK) return e;
+    const int rows = s.batch * s.hq * s.nq;
+    const int blocks = (rows * 32 + 255) / 256;
+    if (s.dv == 64)
+        attend_combine_kernel<64><<<blocks, 256, 0, st>>>(part, out, s.nq, ns, rows);
+    else
+        attend_combine_kernel<128><<<blocks, 256, 0, st>>>(part, out, s.nq, ns, rows);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
 // Attention on the tensor cores with caller-chosen scratch pointers (status

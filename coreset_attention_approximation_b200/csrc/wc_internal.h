@@ -13,6 +13,7 @@ namespace wc {
 constexpr int kMaxBlocksPerUnit = 512;   // select: thread blocks that share one unit
 constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1
 constexpr int kCenterChunk = 1024;       // centring: keys per partial column sum
+constexpr int kAttendFill = 148;         // attention: blocks resident at once (one per SM of a B200)
 // Row of a C1 partial sum: O[0 .. dv), l, m, two unused floats (rows 16-byte aligned).
 constexpr int c1_row(int dv) { return dv + 4; }
 constexpr int kWsAlign = 256;
@@ -49,6 +50,7 @@ struct WsLayout {
     size_t cdot;      // double[units][n]       <k_i, mean>
     size_t bias;      // float[units * bins][stride]  -beta log2(e) <k_i, mean> per bin, padded
     size_t shift;     // double[units * bins]   M = max_i beta |k_i|^2 per bin unit (the factor's shift)
+    size_t apart;     // float[B * hq][splits][nq][c1_row(dv)]  key-split attention rows (few queries only)
     size_t scratch_end;
     // room for outputs that wc_forward keeps in the workspace when not given
     size_t piv, rank, f, ks, w;
@@ -99,6 +101,10 @@ wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st);
 
 // Tensor-core path (bf16 inputs, d and dv in {64, 128}).
 bool tc_supported(const Shape& s);
+// tensor-core attention: splits of the coreset when few query tiles would leave
+// SMs idle (1 = none), and the floats of their partial rows in the workspace
+int attend_splits(const Shape& s);
+size_t attend_split_floats(const Shape& s);
 wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K, const void* V,
                                    const int32_t* rank, char* ws, cudaStream_t st);
 wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,

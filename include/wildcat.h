@@ -95,7 +95,13 @@ typedef struct {
     int32_t batch;    /* B >= 1, B * hq <= 65535 */
     int32_t hq;       /* query heads, a multiple of hkv */
     int32_t hkv;      /* key/value heads >= 1 */
-    int32_t n_k;      /* keys per head, 1 <= n_k <= 2^26 */
+    int32_t n_k;      /* keys per head, 1 <= n_k <= 2^26.  The selection keeps a
+                         unit's residual diagonal in the shared memory of blocks
+                         that run at the same time, which bounds the keys of one
+                         unit (one bin with bins) to what the GPU holds at once:
+                         about 3.6 million on a B200 (148 SMs x ~24.8k rows);
+                         beyond, wc_select / wc_forward return WC_ERR_UNSUPPORTED
+                         before the selection launches */
     int32_t n_q;      /* queries per head >= 0 */
     int32_t d;        /* key/query width, a multiple of 8, 8..256 */
     int32_t dv;       /* value width, a multiple of 8, 8..256 */

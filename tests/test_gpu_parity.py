@@ -12,7 +12,7 @@ import torch
 import oracle
 from coreset_attention_approximation_b200 import wildcat
 from coreset_attention_approximation_b200.workloads import WORKLOADS, make_inputs
-from parity import TOL_OUT, compare, rel_err, run_gpu
+from parity import TOL_OUT, compare, factor_shift, rel_err, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -84,6 +84,26 @@ def test_rank_deficient_keys_stop_and_reproduce_exact_attention():
     assert rel_err(res["out"][0, 0].numpy(), ex) <= 1e-4
 
 
+def test_split_attention_with_empty_splits():
+    """bf16 keys with 6 distinct rows and r = 512: the selection stops at rank
+    6, so of the attention's four key splits (two query heads, one query tile
+    each) only the first holds coreset rows; the combined rows are still exact
+    attention."""
+    g = torch.Generator().manual_seed(3)
+    m, n, d, dv = 6, 1024, 64, 64
+    base = torch.randn(m, d, generator=g, dtype=torch.float64) * 0.25
+    idx = torch.randint(0, m, (n,), generator=g)
+    idx[:m] = torch.arange(m)
+    K = base[idx][None, None].to(torch.bfloat16).contiguous()
+    V = torch.randn(1, 1, n, dv, generator=g, dtype=torch.float64).to(torch.bfloat16)
+    Q = (torch.randn(1, 2, 33, d, generator=g, dtype=torch.float64) * 0.25).to(torch.bfloat16)
+    res = run_gpu(Q, K, V, 512, seed=1)
+    assert int(res["rank"][0, 0]) == m
+    for h in range(2):
+        ex = oracle.exact_attention(Q[0, h], K[0, 0], V[0, 0], 1.0 / np.sqrt(d))
+        assert rel_err(res["out"][0, h].numpy(), ex) <= 2e-3
+
+
 def test_all_keys_equal_gives_mean_of_values():
     n, d, dv = 256, 64, 64
     K = torch.full((1, 1, n, d), 0.05, dtype=torch.bfloat16)
@@ -133,38 +153,52 @@ def test_wait_timeout_is_reported_and_context_survives():
     compare(*make_inputs(w), w.r, seed=0)
 
 
-def test_full_long_workload_prefix_and_properties():
+def test_full_long_workload_head0_and_properties():
     """The bench workload (long: 8 heads, n = 131072, r = 2048) in the bench's
-    launch configuration.  Pivot prefix of head 0 against the oracle (steps
-    0..127), and properties that hold at any size on every head."""
+    launch configuration.  Head 0 in full against the oracle: every pivot
+    (replayed only inside the 1e-6 CDF window), the factor, the weights, and
+    sampled outputs computed by the oracle from its own weights; on every head,
+    properties that hold at any size."""
     w = WORKLOADS["long"]
     Q, K, V = make_inputs(w)
     res = run_gpu(Q, K, V, w.r, seed=0)
     piv, rank = res["piv"].numpy(), res["rank"].numpy()
     assert np.all(rank == w.r)
     beta = 1.0 / np.sqrt(w.d)
-    pre = oracle.rpcholesky(K[0, 0], 128, beta, seed=0, unit=0, replay_piv=piv[0, 0, :128], replay_rank=128)
-    assert pre["failed_step"] == -1
-    F = res["F"]
+    K0 = K[0, 0].double().numpy()
+    sel = oracle.rpcholesky(K0, w.r, beta, seed=0, unit=0, replay_piv=piv[0, 0], replay_rank=w.r)
+    assert sel["failed_step"] == -1 and sel["rank"] == w.r, sel["fail_margin"]
+    assert np.array_equal(sel["piv"], piv[0, 0])
+    # the factor, 256 columns at a time (the library's F is the oracle's times exp(-M/2))
+    scale = np.exp(-factor_shift(K0, beta) / 2)
+    Fo = sel.pop("F")
+    den = float(np.max(np.abs(Fo))) * scale
+    worst = 0.0
+    for c0 in range(0, w.r, 256):
+        g = res["F"][0, 0, c0:c0 + 256, :w.n_k].double().numpy().T
+        worst = max(worst, float(np.max(np.abs(g - Fo[:, c0:c0 + 256] * scale))))
+    del Fo
+    assert worst / den <= 1e-5
+    Wo = oracle.nystrom_weights(K0, V[0, 0], piv[0, 0], w.r, beta)
+    assert rel_err(res["W"][0, 0].numpy(), Wo) <= 2e-3
     rng = np.random.default_rng(0)
+    qs = rng.choice(w.n_q, 256, replace=False)
+    out_o = oracle.coreset_attend(Q[0, 0, qs], K0[piv[0, 0]], Wo, beta)
+    assert rel_err(res["out"][0, 0, qs].numpy(), out_o) <= TOL_OUT[torch.bfloat16]
+    F = res["F"]
     for h in range(w.hkv):
         p = piv[0, h]
         assert len(set(p.tolist())) == w.r
         L = F[0, h][:, p].numpy().T                              # L[a, c] = F[c, piv[a]]
         assert np.all(np.triu(L, 1) == 0.0) and np.all(np.diag(L) > 0.0)
-        # F F^T reproduces H on sampled pivot rows
+        # F F^T reproduces the shifted kernel exp(beta K K^T - M) on sampled pivot rows
         Kh = K[0, h].double().numpy()
-        M = beta * np.max(np.sum(Kh * Kh, axis=1))   # F is the factor of exp(beta K K^T - M)
+        M = factor_shift(Kh, beta)
         for a in rng.choice(w.r, 4, replace=False):
             i = rng.choice(w.n_k, 64, replace=False)
             Hrow = np.exp(beta * Kh[i] @ Kh[p[a]] - M)
             FFt = F[0, h][:, i].double().numpy().T @ L[a].astype(np.float64)
             assert rel_err(FFt, Hrow) <= 1e-4
-    # outputs of sampled queries of head 0 from the GPU's coreset and weights
-    qs = rng.choice(w.n_q, 64, replace=False)
-    k = int(rank[0, 0])
-    out_o = oracle.coreset_attend(Q[0, 0, qs], res["Ks"][0, 0, :k], res["W"][0, 0, :k], beta)
-    assert rel_err(res["out"][0, 0, qs].numpy(), out_o) <= TOL_OUT[torch.bfloat16]
 
 
 def test_running_max_rescale_large_dynamic_range():
@@ -227,3 +261,36 @@ def test_host_pipeline_matches_forward(bins):
     pipe.run([(*pinned[2], outs[0])])
     assert pipe.wait() == 0
     assert torch.equal(outs[0], outs[2])
+
+
+def test_maximum_coreset_size():
+    """r = 4096, the largest coreset the library takes, on keys whose kernel
+    stays full rank (unit directions at norm 6, d = 64: diagonally dominant),
+    so every one of the 4096 steps runs; 6000 keys leave unchosen mass, as in
+    any real use."""
+    w = WORKLOADS["vit"].replace(batch=1, hq=2, hkv=1, n_k=6000, n_q=200, r=4096)
+    Q, K, V = make_inputs(w, seed=41)
+    g = torch.Generator().manual_seed(41)
+    K = (torch.nn.functional.normalize(torch.randn(K.shape, generator=g, dtype=torch.float64), dim=-1) * 6.0).to(K.dtype)
+    compare(Q, K, V, w.r, seed=41, tol_w=2e-3)
+    assert int(run_gpu(Q, K, V, w.r, seed=41)["rank"][0, 0]) == w.r
+
+
+def test_many_keys_in_one_unit():
+    """3,000,037 keys in one unit (293 co-resident blocks of 10240 rows, a
+    ragged last block), the whole path against the oracle."""
+    w = WORKLOADS["vit"].replace(batch=1, hq=2, hkv=1, n_k=3_000_037, n_q=300, r=16)
+    compare(*make_inputs(w, seed=43), w.r, seed=43, tol_w=2e-3)
+
+
+def test_keys_beyond_the_coresident_limit_are_refused():
+    """The select keeps a unit's residual diagonal in the shared memory of
+    co-resident blocks; beyond what the GPU holds at once (about 3.6 million
+    keys a unit on 148 SMs) it returns WC_ERR_UNSUPPORTED without launching."""
+    w = WORKLOADS["vit"].replace(batch=1, hq=1, hkv=1, n_k=4_194_341, n_q=0, r=4)
+    dev = torch.device("cuda")
+    K = torch.zeros(1, 1, w.n_k, w.d, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(wildcat.WildcatError) as e:
+        wildcat.select(K, w.r, seed=0)
+    assert e.value.code == 4
+    torch.cuda.synchronize()
