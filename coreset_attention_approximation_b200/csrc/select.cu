@@ -6,6 +6,12 @@
 // the exponential kernel matrix whose pivot at every step is drawn from the
 // diagonal of the current residual matrix.
 //
+// The factorisation runs on exp(beta K K^T - M), M = max_i beta |k_i|^2 over
+// the unit: the kernel times a positive constant, so the pivot draws (ratios of
+// the residual diagonal) and the stop rule (relative to the diagonal's
+// maximum, now 1) are unchanged, every entry is at most 1 and the fp32 factor
+// cannot overflow; F is the unshifted factor times exp(-M / 2).
+//
 // Design (B200): each (batch, kv-head) unit owns C thread blocks; block c owns
 // a contiguous slice of rows (keys).  The residual diagonal of the slice stays
 // in shared memory in fp64 for the whole run.  A step is
@@ -16,8 +22,8 @@
 //      pivot s_j and its residual through the unit's sync slot;
 //   3. every block streams, for its rows i, the transposed keys Kt[:, i] and
 //      the factor columns F[0..j), i (both laid out with i contiguous, so a
-//      warp reads 512 contiguous bytes per column) and computes
-//        F[j, i] = (exp(beta <k_i, k_s>) - sum_c F[c, i] F[c, s]) / sqrt(d_s)
+//      warp reads 256 contiguous bytes of each F column) and computes
+//        F[j, i] = (exp(beta <k_i, k_s> - M) - sum_c F[c, i] F[c, s]) / sqrt(d_s)
 //      with fp32 products summed in chunks of eight into fp64, then downdates
 //      its residual diagonal and publishes its new slice sum;
 //   4. a bounded barrier among the unit's blocks closes the step.
@@ -545,15 +551,23 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
         return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
     }
     // blocks of a unit wait on each other: co-resident waves, cooperative launch
+    // (the launch attribute form, which stream capture into a CUDA graph takes)
     const int per_wave = (int)(cap / C);
     if (per_wave < 1) return WC_ERR_UNSUPPORTED;
     for (int u0 = 0; u0 < s.units; u0 += per_wave) {
         a.unit0 = u0;
         const int nu = s.units - u0 < per_wave ? s.units - u0 : per_wave;
-        void* args[] = {&a};
-        if (cudaLaunchCooperativeKernel((const void*)kern, dim3(nu * C), dim3(kThreads), args, smem, st) !=
-            cudaSuccess)
-            return WC_ERR_CUDA;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(nu * C);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return WC_ERR_CUDA;
     }
     return WC_OK;
 }

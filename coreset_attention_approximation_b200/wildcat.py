@@ -222,6 +222,42 @@ def forward_host(Q, K, V, r, seed=0, *, device="cuda", ws=None, stream=None, **k
     return out
 
 
+class ForwardGraph:
+    """wc_forward captured once into a CUDA graph, then replayed: repeated
+    forward passes over the same device buffers cost one graph launch instead
+    of the path's kernel launches and memsets.  Refill Q, K, V in place (for
+    example with copy_) before each `replay()`; the outputs (out, piv, rank, F,
+    Ks, W) are overwritten in place and returned."""
+
+    def __init__(self, Q, K, V, r, seed=0, *, ws=None, outputs=None, **kw):
+        self.Q, self.K, self.V = Q, K, V
+        self.shape = shape_of(Q, K, V, r, seed=seed, **kw)
+        self.ws = workspace(self.shape, K.device) if ws is None else ws
+        o = dict(outputs or {})
+        if any(k not in o for k in ("piv", "rank", "F", "Ks", "W")):
+            for k, v in _outputs(self.shape, K.device, K.dtype).items():
+                o.setdefault(k, v)
+        o.setdefault("out", torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], self.shape.dv, dtype=torch.float32,
+                                        device=K.device))
+        self.outputs = o
+        # one eager pass first: function attributes and tensor maps are set up outside the capture
+        self._launch(torch.cuda.current_stream(K.device))
+        torch.cuda.current_stream(K.device).synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._launch(torch.cuda.current_stream(K.device))
+
+    def _launch(self, stream):
+        o = self.outputs
+        _check(lib().wc_forward(ctypes.byref(self.shape), _ptr(self.Q), _ptr(self.K), _ptr(self.V), _ptr(o["out"]),
+                                _ptr(o["piv"]), _ptr(o["rank"]), _ptr(o["F"]), _ptr(o["Ks"]), _ptr(o["W"]),
+                                _ptr(self.ws), self.ws.numel(), _stream(stream)), "wc_forward")
+
+    def replay(self):
+        self.graph.replay()
+        return self.outputs
+
+
 class HostPipeline:
     """Forward passes over a sequence of host batches, with the copies
     overlapped: batch i+1's host-to-device copy and batch i-1's device-to-host
