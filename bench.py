@@ -85,6 +85,13 @@ class ClockSampler:
         self.proc = None
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
 
+    def _lines(self):
+        try:
+            with open(self.file.name) as f:
+                return sum(1 for line in f if line.strip())
+        except OSError:
+            return 0
+
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
@@ -92,10 +99,19 @@ class ClockSampler:
                  "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        # the first sample lands before the timed region starts (nvidia-smi takes a moment to come up)
+        t0 = time.time()
+        while self.proc is not None and self._lines() == 0 and time.time() - t0 < 5.0:
+            time.sleep(0.02)
+        self.n_enter = self._lines()
         return self
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            # a short timed region still gets the sample that follows it
+            t0 = time.time()
+            while self._lines() <= self.n_enter and time.time() - t0 < 1.0:
+                time.sleep(0.02)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)

@@ -38,6 +38,9 @@
 namespace wc {
 namespace {
 
+// threads per block: 256 (2 blocks per SM), or 128 (4 per SM) where the units
+// are too many for 2 blocks per SM to give each enough of them (binned
+// selections); shared memory is planned for the larger
 constexpr int kThreads = 256;
 // rows per thread per pass (one float2 of F): with about 14 rows of a block's
 // slice per thread, 2-row groups keep the threads of a block evenly loaded
@@ -91,6 +94,7 @@ struct Bcast {
 // Inclusive scan over the block of one double per thread (fixed order,
 // deterministic); writes each thread's inclusive value to scan[tid] and
 // returns the block total.
+template <int NT>
 __device__ double block_scan(double v, double* scan) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -98,29 +102,30 @@ __device__ double block_scan(double v, double* scan) {
         const double y = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += y;
     }
-    __shared__ double wtot[kThreads / 32];
+    __shared__ double wtot[NT / 32];
     if (lane == 31) wtot[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        double w = lane < kThreads / 32 ? wtot[lane] : 0.0;
+        double w = lane < NT / 32 ? wtot[lane] : 0.0;
 #pragma unroll
-        for (int o = 1; o < kThreads / 32; o <<= 1) {
+        for (int o = 1; o < NT / 32; o <<= 1) {
             const double y = __shfl_up_sync(0xffffffffu, w, o);
             if (lane >= o) w += y;
         }
-        if (lane < kThreads / 32) wtot[lane] = w;
+        if (lane < NT / 32) wtot[lane] = w;
     }
     __syncthreads();
     if (warp > 0) v += wtot[warp - 1];
     scan[threadIdx.x] = v;
-    const double total = wtot[kThreads / 32 - 1];
+    const double total = wtot[NT / 32 - 1];
     __syncthreads();
     return total;
 }
 
 // Contiguous chunk of the slice that thread `t` sums for the scans.
+template <int NT>
 __device__ __forceinline__ void chunk_of(int t, int mlen, int* lo, int* hi) {
-    const int q = (mlen + kThreads - 1) / kThreads;
+    const int q = (mlen + NT - 1) / NT;
     *lo = min(mlen, t * q);
     *hi = min(mlen, *lo + q);
 }
@@ -227,8 +232,8 @@ __device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, 
 
 // T: element type of K; TK: of the transposed copy that every step streams
 // (T, or fp32 when the keys are centred).
-template <typename T, typename TK>
-__global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArgs a) {
+template <typename T, typename TK, int NT>
+__global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int tid = threadIdx.x;
     const int unit = a.unit0 + blockIdx.x / a.C;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
 
     double* dg = reinterpret_cast<double*>(smem);
     double* scan = dg + a.m;
-    double* bsum = scan + kThreads;
+    double* bsum = scan + kThreads;  // the scan array is planned for the larger block
     double* ks = bsum + kMaxBlocksPerUnit;
     float* fs = reinterpret_cast<float*>(ks + d);
     unsigned char* ispiv = reinterpret_cast<unsigned char*>(fs + r);
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     // ---- initial residual in the log domain, beta |k_i|^2 (centred: k_i - kbar, in
     // fp64, the transposed copy stored as fp32); transpose the slice
     double lmax = 0.0;
-    for (int il = tid; il < ng * kGroup; il += kThreads) {
+    for (int il = tid; il < ng * kGroup; il += NT) {
         const int i = r0 + il;
         if (il < mlen) {
             const T* krow = K + (size_t)i * d;
@@ -299,14 +304,14 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             alive = false;
         }
     }
-    for (int il = tid; il < mlen; il += kThreads) dg[il] = exp(dg[il] - shift);
+    for (int il = tid; il < mlen; il += NT) dg[il] = exp(dg[il] - shift);
     __syncthreads();  // the scan chunks below span rows that other threads initialised
     {
         int lo, hi;
-        chunk_of(tid, mlen, &lo, &hi);
+        chunk_of<NT>(tid, mlen, &lo, &hi);
         double sum = 0.0;
         for (int il = lo; il < hi; ++il) sum += dg[il];
-        const double tot = block_scan(sum, scan);
+        const double tot = block_scan<NT>(sum, scan);
         if (tid == 0) part[blk] = tot;
     }
     if (alive) alive = unit_barrier(&us->bar, a.C, 2, a.timeout_ns, status, &bc.ok);
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         // 1. which block's slice holds t = u_j * sum(d): the unit's block sums
         // come into shared memory in parallel, then one thread adds them in
         // block order
-        for (int c = tid; c < a.C; c += kThreads) bsum[c] = __ldcg(pj + c);
+        for (int c = tid; c < a.C; c += NT) bsum[c] = __ldcg(pj + c);
         __syncthreads();
         if (tid == 0) {
             double total = 0.0;
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
                 }
                 bc.tau = tau;
             }
-            bc.tstar = kThreads;
+            bc.tstar = NT;
         }
         __syncthreads();
         if (bc.stop) { final_rank = j; break; }
@@ -356,11 +361,11 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
             const double base = bc.base, tau = bc.tau;
             if (base + scan[tid] > tau) atomicMin(&bc.tstar, tid);
             __syncthreads();
-            if (tid == 0 && bc.tstar == kThreads) bc.tstar = kThreads - 1;  // rounding guard
+            if (tid == 0 && bc.tstar == NT) bc.tstar = NT - 1;  // rounding guard
             __syncthreads();
             if (tid == bc.tstar) {
                 int lo, hi;
-                chunk_of(tid, mlen, &lo, &hi);
+                chunk_of<NT>(tid, mlen, &lo, &hi);
                 double run = tid == 0 ? base : base + scan[tid - 1];
                 int sl = -1;
                 for (int il = lo; il < hi; ++il) {
@@ -403,24 +408,24 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         const double ds = bc.d_s;
 
         // 3. pivot key and F[s, 0..j) into shared memory
-        for (int c = tid; c < d; c += kThreads) ks[c] = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
-        for (int c0 = tid; c0 < j; c0 += 8 * kThreads) {  // 8 loads in flight before the stores
+        for (int c = tid; c < d; c += NT) ks[c] = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
+        for (int c0 = tid; c0 < j; c0 += 8 * NT) {  // 8 loads in flight before the stores
             float v[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const int c = c0 + q * kThreads;
+                const int c = c0 + q * NT;
                 v[q] = c < j ? ld_cg_f32(F + (int64_t)c * ldf + s) : 0.f;
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                if (c0 + q * kThreads < j) fs[c0 + q * kThreads] = v[q];
+                if (c0 + q * NT < j) fs[c0 + q * NT] = v[q];
         }
         __syncthreads();
 
         // 4. column j over this block's rows, and the residual downdate
         const double root = sqrt(ds);
         float* Fj = F + (int64_t)j * ldf;
-        for (int g = tid; g < ng; g += kThreads) {
+        for (int g = tid; g < ng; g += NT) {
             const int il0 = g * kGroup;
             const int i0 = r0 + il0;
             double dot[kGroup], cor[kGroup];
@@ -450,10 +455,10 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
         // 5. new slice sum, then close the step
         {
             int lo, hi;
-            chunk_of(tid, mlen, &lo, &hi);
+            chunk_of<NT>(tid, mlen, &lo, &hi);
             double sum = 0.0;
             for (int il = lo; il < hi; ++il) sum += dg[il];
-            const double tot = block_scan(sum, scan);
+            const double tot = block_scan<NT>(sum, scan);
             if (tid == 0) part[(size_t)((j + 1) & 1) * kMaxBlocksPerUnit + blk] = tot;
         }
         if (!unit_barrier(&us->bar, a.C, (uint32_t)j + 3u, a.timeout_ns, status, &bc.ok)) {
@@ -466,15 +471,90 @@ __global__ void __launch_bounds__(kThreads, 2) rpcholesky_kernel(const SelectArg
     // ---- columns >= rank are zero; piv beyond rank is -1
     for (int jj = final_rank; jj < r; ++jj) {
         float* Fj = F + (int64_t)jj * ldf;
-        for (int g = tid; g < ng; g += kThreads) {
+        for (int g = tid; g < ng; g += NT) {
             const int i0 = r0 + g * kGroup;
             *reinterpret_cast<float2*>(Fj + i0) = make_float2(0.f, 0.f);
         }
     }
     if (blk == 0) {
-        for (int jj = final_rank + tid; jj < r; jj += kThreads) a.piv[(size_t)unit * r + jj] = -1;
+        for (int jj = final_rank + tid; jj < r; jj += NT) a.piv[(size_t)unit * r + jj] = -1;
         if (tid == 0) a.rank[unit] = final_rank;
     }
+}
+
+struct SelectPlan {
+    int C = 0, m = 0;   // blocks per unit, rows per block
+    long cap = 0;       // blocks the GPU holds at once with m rows each
+    int per_sm = 0;     // of those, a SM's
+};
+
+// Most blocks per unit such that every block of the launch is co-resident
+// (they wait on each other), at >= 256 rows per block; else the fewest blocks
+// the shared memory allows, in co-resident waves.
+template <typename T, typename TK, int NT>
+wc_status plan_select(const Shape& s, int nsm, int max_smem, int m_max, SelectPlan* p) {
+    auto kern = rpcholesky_kernel<T, TK, NT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem - 1024) != cudaSuccess)
+        return WC_ERR_CUDA;
+    auto blocks_per_sm = [&](int m) {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, NT, select_smem_bytes(m, s.r, s.d)) != cudaSuccess)
+            return 0;
+        return b;
+    };
+    auto rows_for = [&](int C) { return ((s.n + C - 1) / C + kRowAlign - 1) / kRowAlign * kRowAlign; };
+    const int c_min = (s.n + m_max - 1) / m_max;
+    int c_hi = (s.n + 255) / 256;
+    if (c_hi > kMaxBlocksPerUnit) c_hi = kMaxBlocksPerUnit;
+    if (c_hi < c_min) c_hi = c_min;
+    int m = rows_for(c_min);
+    int bps = blocks_per_sm(m);
+    for (int c = c_hi; c > c_min; --c) {
+        const int mc = rows_for(c);
+        const int ce = (s.n + mc - 1) / mc;
+        const int bc = blocks_per_sm(mc);
+        if ((long)s.units * ce <= (long)nsm * bc) {
+            m = mc;
+            bps = bc;
+            break;
+        }
+    }
+    p->m = m;
+    p->C = (s.n + m - 1) / m;
+    p->per_sm = bps;
+    p->cap = (long)nsm * bps;
+    return WC_OK;
+}
+
+template <typename T, typename TK, int NT>
+wc_status run_select(const Shape& s, const SelectPlan& p, SelectArgs a, char* ws, cudaStream_t st) {
+    auto kern = rpcholesky_kernel<T, TK, NT>;
+    const size_t smem = select_smem_bytes(p.m, s.r, s.d);
+    if (p.C == 1) {
+        a.unit0 = 0;
+        kern<<<s.units, NT, smem, st>>>(a);
+        return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+    }
+    // blocks of a unit wait on each other: co-resident waves, cooperative launch
+    // (the launch attribute form, which stream capture into a CUDA graph takes)
+    const int per_wave = (int)(p.cap / p.C);
+    if (per_wave < 1) return WC_ERR_UNSUPPORTED;
+    for (int u0 = 0; u0 < s.units; u0 += per_wave) {
+        a.unit0 = u0;
+        const int nu = s.units - u0 < per_wave ? s.units - u0 : per_wave;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(nu * p.C);
+        cfg.blockDim = dim3(NT);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
 }
 
 template <typename T, typename TK>
@@ -493,42 +573,23 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     int m_max = (int)(((size_t)max_smem - fixed) / 9) / kRowAlign * kRowAlign;
     m_max = m_max > (1 << 20) ? (1 << 20) : m_max;
 
-    auto kern = rpcholesky_kernel<T, TK>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem - 1024) != cudaSuccess)
-        return WC_ERR_CUDA;
-    auto blocks_per_sm = [&](int m) {
-        int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, select_smem_bytes(m, s.r, s.d)) !=
-            cudaSuccess)
-            return 0;
-        return b;
+    // 256-thread blocks, unless the launch is one co-resident wave either way
+    // and 128-thread blocks leave the busiest SM fewer rows: with 2 blocks per
+    // SM, units that are many and short (bins) leave SMs idle
+    SelectPlan p256, p128;
+    wc_status e = plan_select<T, TK, 256>(s, nsm, max_smem, m_max, &p256);
+    if (e != WC_OK) return e;
+    if ((e = plan_select<T, TK, 128>(s, nsm, max_smem, m_max, &p128)) != WC_OK) return e;
+    auto one_wave = [&](const SelectPlan& p) { return p.C > 1 && (long)s.units * p.C <= p.cap; };
+    auto sm_rows = [&](const SelectPlan& p) {
+        const long blocks = (long)s.units * p.C;
+        const long per_sm = (blocks + nsm - 1) / nsm;
+        return (long)p.m * (per_sm < p.per_sm ? per_sm : p.per_sm);
     };
-    auto rows_for = [&](int C) { return ((s.n + C - 1) / C + kRowAlign - 1) / kRowAlign * kRowAlign; };
-
-    // Most blocks per unit such that every block of the launch is co-resident
-    // (they wait on each other), at >= 256 rows per block; else the fewest
-    // blocks the shared memory allows, in co-resident waves.
-    const int c_min = (s.n + m_max - 1) / m_max;
-    int c_hi = (s.n + 255) / 256;
-    if (c_hi > kMaxBlocksPerUnit) c_hi = kMaxBlocksPerUnit;
-    if (c_hi < c_min) c_hi = c_min;
-    int C = c_min, m = rows_for(c_min);
-    long cap = (long)nsm * blocks_per_sm(m);
-    for (int c = c_hi; c > c_min; --c) {
-        const int mc = rows_for(c);
-        const int ce = (s.n + mc - 1) / mc;
-        const long capc = (long)nsm * blocks_per_sm(mc);
-        if ((long)s.units * ce <= capc) {
-            C = ce;
-            m = mc;
-            cap = capc;
-            break;
-        }
-    }
-    C = (s.n + m - 1) / m;
-    const size_t smem = select_smem_bytes(m, s.r, s.d);
-    if (cap < 1) return WC_ERR_CUDA;
-    if (C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
+    const bool use128 = one_wave(p256) && one_wave(p128) && sm_rows(p128) * 100 < sm_rows(p256) * 97;
+    const SelectPlan& p = use128 ? p128 : p256;
+    if (p.cap < 1) return WC_ERR_CUDA;
+    if (p.C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
 
     SelectArgs a;
     a.K = K; a.piv = piv; a.F = F; a.rank = rank;
@@ -540,36 +601,11 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     a.partials = reinterpret_cast<double*>(ws + L.partials);
     a.status = reinterpret_cast<int*>(ws + L.status);
     a.ldf = s.ldf; a.n = s.n; a.d = s.d; a.r = s.r;
-    a.C = C; a.m = m;
+    a.C = p.C; a.m = p.m;
     a.beta = s.beta; a.eps = s.eps; a.seed = s.seed; a.timeout_ns = s.timeout_ns;
 
     if (cudaMemsetAsync(ws + L.sync, 0, sizeof(UnitSync) * (size_t)s.units, st) != cudaSuccess) return WC_ERR_CUDA;
-
-    if (C == 1) {
-        a.unit0 = 0;
-        kern<<<s.units, kThreads, smem, st>>>(a);
-        return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
-    }
-    // blocks of a unit wait on each other: co-resident waves, cooperative launch
-    // (the launch attribute form, which stream capture into a CUDA graph takes)
-    const int per_wave = (int)(cap / C);
-    if (per_wave < 1) return WC_ERR_UNSUPPORTED;
-    for (int u0 = 0; u0 < s.units; u0 += per_wave) {
-        a.unit0 = u0;
-        const int nu = s.units - u0 < per_wave ? s.units - u0 : per_wave;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(nu * C);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return WC_ERR_CUDA;
-    }
-    return WC_OK;
+    return use128 ? run_select<T, TK, 128>(s, p, a, ws, st) : run_select<T, TK, 256>(s, p, a, ws, st);
 }
 
 // Two blocks meet at a unit barrier that block 1 never reaches: block 0's
