@@ -1,6 +1,9 @@
-"""Builds libwildcat.so (sm_100a) in the package directory with nvcc.
+"""Builds libwildcat.so (sm_100a) in the package directory with nvcc, and its
+bounds-checked twin libwildcat_debug.so (the same sources with
+-DWC_DEBUG_BOUNDS=1: every data-dependent index is checked against its buffer
+and a bad one is recorded as WC_ERR_BOUNDS instead of accessed).
 
-    python -m coreset_attention_approximation_b200.build
+    python -m coreset_attention_approximation_b200.build [--debug]
 """
 
 from __future__ import annotations
@@ -30,17 +33,20 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose: bool = False, jobs: int | None = None) -> str:
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(verbose: bool = False, jobs: int | None = None, debug: bool = False) -> str:
+    objdir = OBJDIR + ("_debug" if debug else "")
+    lib = os.path.join(HERE, "libwildcat_debug.so") if debug else LIB
+    flags = FLAGS + (["-DWC_DEBUG_BOUNDS=1"] if debug else [])
+    os.makedirs(objdir, exist_ok=True)
     include = os.path.join(os.path.dirname(HERE), "include", "wildcat.h")
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [include, __file__]
     objs, procs = [], []
     for src in SOURCES:
         path = os.path.join(CSRC, src)
-        obj = os.path.join(OBJDIR, src.replace(".cu", ".o"))
+        obj = os.path.join(objdir, src.replace(".cu", ".o"))
         objs.append(obj)
         if _stale(obj, [path] + hdrs):
-            cmd = [NVCC, *FLAGS, "-c", path, "-o", obj]
+            cmd = [NVCC, *flags, "-c", path, "-o", obj]
             if verbose:
                 print(" ".join(cmd), flush=True)
             procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -53,13 +59,13 @@ def build(verbose: bool = False, jobs: int | None = None) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed for {failed}")
-    if _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp,
-                        "-lcudart"], check=True)
-        os.replace(tmp, LIB)
-    return LIB
+                        "-lcudart", "-ldl"], check=True)
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose=True))
+    print(build(verbose=True, debug="--debug" in sys.argv[1:]))

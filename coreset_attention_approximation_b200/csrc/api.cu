@@ -1,6 +1,7 @@
 // api.cu — the C ABI (include/wildcat.h): argument checks, workspace layout,
 // and the launch sequences of select, weights, attend and forward.
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <string.h>
 
 #include "wc_common.cuh"
@@ -123,6 +124,14 @@ static wc_status check_ws(const Shape& s, void* ws, size_t ws_bytes, bool forwar
 
 using namespace wc;
 
+namespace {
+// An NVTX range around each entry point, for profilers (no cost without one).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
+
 extern "C" {
 
 int64_t wc_f_ld(int32_t n_k) { return n_k < 1 ? 0 : f_ld(n_k); }
@@ -141,6 +150,7 @@ size_t wc_forward_workspace_bytes(const wc_shape* shape) {
 
 wc_status wc_select(const wc_shape* shape, const void* K, int32_t* piv, float* F, int32_t* rank, void* ws,
                     size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("wc_select");
     Shape s;
     wc_status e = make_shape(shape, &s);
     if (e != WC_OK) return e;
@@ -154,6 +164,7 @@ wc_status wc_select(const wc_shape* shape, const void* K, int32_t* piv, float* F
 
 wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const int32_t* piv, const float* F,
                      const int32_t* rank, void* Ks, float* W, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("wc_weights");
     Shape s;
     wc_status e = make_shape(shape, &s);
     if (e != WC_OK) return e;
@@ -172,6 +183,7 @@ wc_status wc_weights(const wc_shape* shape, const void* K, const void* V, const 
 
 wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const float* W, const int32_t* rank,
                     float* out, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("wc_attend");
     Shape s;
     wc_status e = make_shape(shape, &s);
     if (e != WC_OK) return e;
@@ -184,6 +196,7 @@ wc_status wc_attend(const wc_shape* shape, const void* Q, const void* Ks, const 
 
 wc_status wc_forward(const wc_shape* shape, const void* Q, const void* K, const void* V, float* out, int32_t* piv,
                      int32_t* rank, float* F, void* Ks, float* W, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("wc_forward");
     Shape s;
     wc_status e = make_shape(shape, &s);
     if (e != WC_OK) return e;
@@ -232,6 +245,7 @@ const char* wc_status_string(wc_status status) {
         case WC_ERR_UNSUPPORTED: return "unsupported shape";
         case WC_ERR_WORKSPACE: return "workspace too small";
         case WC_ERR_NUMERIC: return "non-finite value on the device";
+        case WC_ERR_BOUNDS: return "index outside its buffer (debug build)";
     }
     return "unknown status";
 }

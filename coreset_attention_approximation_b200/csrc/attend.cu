@@ -19,6 +19,7 @@ wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const flo
     e.C = W; e.c_stride = (int64_t)s.r * (s.dv + 1); e.ldc = s.dv + 1;
     e.wcol = W + s.dv;
     e.rank = rank;
+    e.status = ws ? reinterpret_cast<int*>(ws + make_layout(s).status) : nullptr;
     e.all_keys = s.bins > 1;  // bins: padded rows carry zero weights, every row of the union counts
     e.out = out;
     e.d = s.d; e.dv = s.dv; e.r = s.r;

@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(kThreads) expmm_simt_kernel(const ExpmmArgs e)
     if (MODE == kExpmmPartial) {
         unit = z;
         a_valid = e.rank[unit];
+        if (!in_bounds(a_valid >= 0 && a_valid <= e.r, e.status)) return;
         split = blockIdx.y;
         b_lo = split * e.split_len;
         b_hi = min(e.b_rows, b_lo + e.split_len);
@@ -38,6 +39,7 @@ __global__ void __launch_bounds__(kThreads) expmm_simt_kernel(const ExpmmArgs e)
         a_valid = e.a_rows;
         b_lo = 0;
         b_hi = e.all_keys ? e.b_rows : e.rank[unit];
+        if (!in_bounds(b_hi >= 0 && b_hi <= e.b_rows, e.status)) return;
     }
     const int a0 = blockIdx.x * BM;
     if (a0 >= a_valid) return;

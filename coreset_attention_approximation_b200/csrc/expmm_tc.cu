@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!kQueries) {
         unit = z;
         a_valid = args.rank[unit];
+        if (!in_bounds(a_valid >= 0 && a_valid <= args.r, args.status)) return;
         split = blockIdx.y;
         b_lo = split * args.split_len;
         b_hi = min(args.b_rows, b_lo + args.split_len);
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         unit = (z / args.hq) * hkv + (z % args.hq) / args.group;
         a_valid = args.a_rows;
         const int b_all = args.all_keys ? args.b_rows : args.rank[unit];
+        if (!in_bounds(b_all >= 0 && b_all <= args.b_rows, args.status)) return;
         split = MODE == kModeAttnSplit ? (int)blockIdx.y : 0;
         b_lo = split * args.split_len;
         b_hi = min(b_all, b_lo + args.split_len);
@@ -610,13 +612,14 @@ constexpr int kPrepWarps = 8;
 
 __global__ void __cluster_dims__(kPrepCluster, 1, 1) __launch_bounds__(kPrepWarps * 32)
     weights_prep_kernel(const float* __restrict__ W, const int32_t* __restrict__ rank, float* sigma, __half* W16,
-                        float* wn, int r, int r_pad, int dv, int all_keys) {
+                        float* wn, int r, int r_pad, int dv, int all_keys, int* status) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     const int q = (int)cluster.block_rank();
     const int u = blockIdx.x / kPrepCluster, lane = threadIdx.x & 31, g = threadIdx.x >> 5;
     const int c = blockIdx.y * 32 + lane;
-    const int k = all_keys ? r : rank[u];
+    int k = all_keys ? r : rank[u];
+    if (!in_bounds(k >= 0 && k <= r, status)) k = 0;   // (no early return: the cluster waits below)
     const float* Wu = W + (size_t)u * r * (dv + 1);
     const int s0 = q * kPrepWarps + g, step = kPrepCluster * kPrepWarps;
     float mx = 0.f;
@@ -653,9 +656,9 @@ __global__ void __cluster_dims__(kPrepCluster, 1, 1) __launch_bounds__(kPrepWarp
 }
 
 wc_status launch_weights_prep(const Shape& s, const float* W, const int32_t* rank, __half* W16, float* sigma,
-                              float* wn, cudaStream_t st) {
+                              float* wn, int* status, cudaStream_t st) {
     weights_prep_kernel<<<dim3(s.units * kPrepCluster, (s.dv + 31) / 32), kPrepWarps * 32, 0, st>>>(
-        W, rank, sigma, W16, wn, s.r, s.r_pad, s.dv, s.bins > 1);
+        W, rank, sigma, W16, wn, s.r, s.r_pad, s.dv, s.bins > 1, status);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -777,7 +780,8 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     __half* W16 = reinterpret_cast<__half*>(ws + Lw.w16);
     float* sigma = reinterpret_cast<float*>(ws + Lw.sigma);
     float* wn = reinterpret_cast<float*>(ws + Lw.wn);
-    if (launch_weights_prep(s, W, rank, W16, sigma, wn, st) != WC_OK) return WC_ERR_CUDA;
+    if (launch_weights_prep(s, W, rank, W16, sigma, wn, reinterpret_cast<int*>(ws + Lw.status), st) != WC_OK)
+        return WC_ERR_CUDA;
     CUtensorMap mA, mB, mC;
     if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
         !make_map(&mB, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BN) ||
@@ -828,7 +832,7 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
 // point that allocates nothing.
 wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, const float* W, const int32_t* rank,
                               float* out, int* status, __half* W16, float* sigma, float* wn, cudaStream_t st) {
-    if (launch_weights_prep(s, W, rank, W16, sigma, wn, st) != WC_OK) return WC_ERR_CUDA;
+    if (launch_weights_prep(s, W, rank, W16, sigma, wn, status, st) != WC_OK) return WC_ERR_CUDA;
     CUtensorMap mA, mB, mC;
     if (!make_map(&mA, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.batch * s.hq * s.nq, BM) ||
         !make_map(&mB, Ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, s.d, (uint64_t)s.units * s.r, BN) ||

@@ -406,6 +406,10 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
         if (bc.stop) { final_rank = j; break; }
         const int s = bc.s;
         const double ds = bc.d_s;
+        if (!in_bounds(s >= 0 && s < n, status)) {  // every block reads the same s: all stop here
+            final_rank = j;
+            break;
+        }
 
         // 3. pivot key and F[s, 0..j) into shared memory
         for (int c = tid; c < d; c += NT) ks[c] = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
@@ -428,6 +432,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
         for (int g = tid; g < ng; g += NT) {
             const int il0 = g * kGroup;
             const int i0 = r0 + il0;
+            if (!in_bounds(i0 + kGroup <= ldf, status)) continue;
             double dot[kGroup], cor[kGroup];
             key_dots<TK>(Kt + i0, ldf, d, ks, dot);
             correction(F + i0, ldf, j, fs, cor);

@@ -20,6 +20,24 @@ __device__ __forceinline__ void record_status(int* status, int code) {
     atomicCAS(status, 0, code);
 }
 
+// Bounds checks of data-dependent indices (pivots, ranks), compiled in with
+// -DWC_DEBUG_BOUNDS=1 (libwildcat_debug.so): a failed check records
+// WC_ERR_BOUNDS and the caller skips the access.  In the release build every
+// check is `true` and costs nothing.
+#ifndef WC_DEBUG_BOUNDS
+#define WC_DEBUG_BOUNDS 0
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok, int* status) {
+#if WC_DEBUG_BOUNDS
+    if (!ok && status) record_status(status, WC_ERR_BOUNDS);
+    return ok;
+#else
+    (void)ok;
+    (void)status;
+    return true;
+#endif
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

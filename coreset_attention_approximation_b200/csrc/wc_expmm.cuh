@@ -17,6 +17,7 @@ struct ExpmmArgs {
     const void* C;  int64_t c_stride; int ldc;      // value rows (dtype, or fp32 W)
     const float* wcol;                              // rownorm: W[:, dv] with row stride ldc
     const int32_t* rank;                            // valid coreset rows per unit
+    int* status;                                    // device status word (bounds checks of rank)
     int all_keys;                                   // rownorm: every one of the b_rows rows counts
     const float* bias;                              // partial: per-key logit bias (log2 units) or null
     int bias_stride;                                // floats per unit of bias

@@ -23,12 +23,15 @@ namespace {
 template <typename T>
 __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict__ piv,
                               const float* __restrict__ F, const int32_t* __restrict__ rank, T* Ks,
-                              float* Lg, int n, int d, int r, int64_t ldf, int bins) {
+                              float* Lg, int n, int d, int r, int64_t ldf, int bins, int* status) {
     const int a = blockIdx.x, u = blockIdx.y;
-    const int k = rank[u];
+    int k = rank[u];
+    if (!in_bounds(k >= 0 && k <= r, status)) k = 0;
     const int base = (u % bins) * n;  // the bin's first key within the caller's unit
-    const int p = a < k ? piv[(size_t)u * r + a] - base : -1;
-    const int pk = p >= 0 ? p : (bins > 1 && k > 0 ? piv[(size_t)u * r] - base : -1);
+    int p = a < k ? piv[(size_t)u * r + a] - base : -1;
+    int pk = p >= 0 ? p : (bins > 1 && k > 0 ? piv[(size_t)u * r] - base : -1);
+    if (!in_bounds(a >= k || (p >= 0 && p < n), status)) p = -1;
+    if (!in_bounds(pk < n && (pk >= 0 || a >= k), status)) pk = -1;
     T* ks = Ks + ((size_t)u * r + a) * d;
     for (int c = threadIdx.x; c < d; c += blockDim.x)
         ks[c] = pk >= 0 ? K[((size_t)u * n + pk) * d + c] : T(0.f);
@@ -47,13 +50,15 @@ __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict
 __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t* __restrict__ rank, double* Ct,
                                 int nsplit, int r, int dv, const int32_t* __restrict__ piv,
                                 const double* __restrict__ cdot, const double* __restrict__ kk, int bins, int n_all,
-                                double beta, const double* __restrict__ shift) {
+                                double beta, const double* __restrict__ shift, int* status) {
     const int a = blockIdx.x, u = blockIdx.y;
-    if (a >= rank[u]) return;
+    if (a >= rank[u] || !in_bounds(rank[u] <= r, status)) return;
     double rho = -shift[u];
     if (cdot) {
         const int uc = u / bins;  // the caller's unit
-        rho += beta * (kk[uc] - cdot[(size_t)uc * n_all + piv[(size_t)u * r + a]]);
+        const int p = piv[(size_t)u * r + a];
+        if (!in_bounds(p >= 0 && p < n_all, status)) return;
+        rho += beta * (kk[uc] - cdot[(size_t)uc * n_all + p]);
     }
     const int w = c1_row(dv), wcols = dv + 1;
     const float* part = c1part + (size_t)u * nsplit * r * w;
@@ -89,7 +94,8 @@ constexpr int kTrsmThreads = 256;
 template <int NC>
 __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restrict__ Lg,
                                                            const int32_t* __restrict__ rank,
-                                                           const double* __restrict__ Ct, float* W, int r, int dv) {
+                                                           const double* __restrict__ Ct, float* W, int r, int dv,
+                                                           int* status) {
     extern __shared__ double sm_d[];
     double* Y = sm_d;                                        // [r][NC]
     double* rinv = Y + (size_t)r * NC;                       // [kTB] 1 / L_ii of the diagonal block
@@ -98,7 +104,8 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
     const int wcols = dv + 1;
     const int c0 = blockIdx.x * NC;
     const int nc = min(NC, wcols - c0);
-    const int k = rank[u];
+    int k = rank[u];
+    if (!in_bounds(k >= 0 && k <= r, status)) k = 0;
     const float* L = Lg + (size_t)u * r * r;
     const double* C = Ct + (size_t)u * wcols * r;
     float* Wu = W + (size_t)u * r * wcols;
@@ -230,11 +237,12 @@ size_t trsm_smem(int r) {
 
 template <int NC>
 wc_status launch_trsm_t(const Shape& s, const float* Lg, const int32_t* rank, const double* Ct, float* W,
-                        cudaStream_t st) {
+                        int* status, cudaStream_t st) {
     const size_t smem = trsm_smem<NC>(s.r);
     if (cudaFuncSetAttribute(trsm_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return WC_ERR_CUDA;
-    trsm_kernel<NC><<<dim3((s.dv + 1 + NC - 1) / NC, s.units), kTrsmThreads, smem, st>>>(Lg, rank, Ct, W, s.r, s.dv);
+    trsm_kernel<NC><<<dim3((s.dv + 1 + NC - 1) / NC, s.units), kTrsmThreads, smem, st>>>(Lg, rank, Ct, W, s.r, s.dv,
+                                                                                        status);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -244,14 +252,16 @@ wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const
                         void* Ks, char* ws, cudaStream_t st) {
     const WsLayout L = make_layout(s);
     float* Lg = reinterpret_cast<float*>(ws + L.lg);
+    int* status = reinterpret_cast<int*>(ws + L.status);
     dim3 grid(s.r, s.units);
     if (s.dtype == WC_BF16)
         gather_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(K), piv, F, rank,
                                                            static_cast<__nv_bfloat16*>(Ks), Lg, s.n, s.d, s.r,
-                                                           s.ldf, s.bins);
+                                                           s.ldf, s.bins, status);
     else
         gather_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(K), piv, F, rank,
-                                                   static_cast<float*>(Ks), Lg, s.n, s.d, s.r, s.ldf, s.bins);
+                                                   static_cast<float*>(Ks), Lg, s.n, s.d, s.r, s.ldf, s.bins,
+                                                   status);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -265,6 +275,7 @@ wc_status launch_coreset_values(const Shape& s, const void* Ks, const void* K, c
     e.C = V; e.c_stride = (int64_t)s.n * s.dv; e.ldc = s.dv;
     e.wcol = nullptr;
     e.rank = rank;
+    e.status = reinterpret_cast<int*>(ws + L.status);
     e.out = ws + L.c1part;
     e.d = s.d; e.dv = s.dv; e.r = s.r;
     e.nsplit = s.nsplit; e.split_len = kSplitKeys;
@@ -282,19 +293,20 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
                        cudaStream_t st) {
     const WsLayout L = make_layout(s);
     double* Ct = reinterpret_cast<double*>(ws + L.y);
+    int* status = reinterpret_cast<int*>(ws + L.status);
     merge_c1_kernel<<<dim3(s.r, s.units), 160, 0, st>>>(
         reinterpret_cast<const float*>(ws + L.c1part), rank, Ct, s.nsplit, s.r, s.dv, piv,
         s.center ? reinterpret_cast<const double*>(ws + L.cdot) : nullptr,
         s.center ? reinterpret_cast<const double*>(ws + L.kk) : nullptr, s.bins, s.n_all, s.beta,
-        reinterpret_cast<const double*>(ws + L.shift));
+        reinterpret_cast<const double*>(ws + L.shift), status);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
     // as many right-hand sides per block as shared memory holds for this r
     const float* Lg = reinterpret_cast<const float*>(ws + L.lg);
     constexpr size_t kMax = 232448;
-    if (trsm_smem<8>(s.r) <= kMax) return launch_trsm_t<8>(s, Lg, rank, Ct, W, st);
-    if (trsm_smem<4>(s.r) <= kMax) return launch_trsm_t<4>(s, Lg, rank, Ct, W, st);
-    if (trsm_smem<2>(s.r) <= kMax) return launch_trsm_t<2>(s, Lg, rank, Ct, W, st);
-    if (trsm_smem<1>(s.r) <= kMax) return launch_trsm_t<1>(s, Lg, rank, Ct, W, st);
+    if (trsm_smem<8>(s.r) <= kMax) return launch_trsm_t<8>(s, Lg, rank, Ct, W, status, st);
+    if (trsm_smem<4>(s.r) <= kMax) return launch_trsm_t<4>(s, Lg, rank, Ct, W, status, st);
+    if (trsm_smem<2>(s.r) <= kMax) return launch_trsm_t<2>(s, Lg, rank, Ct, W, status, st);
+    if (trsm_smem<1>(s.r) <= kMax) return launch_trsm_t<1>(s, Lg, rank, Ct, W, status, st);
     return WC_ERR_UNSUPPORTED;
 }
 

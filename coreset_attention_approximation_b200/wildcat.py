@@ -20,7 +20,8 @@ LIB_PATH = os.path.join(HERE, "libwildcat.so")
 
 WC_F32, WC_BF16 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "CUDA error", 3: "device-side wait timed out",
-          4: "unsupported shape", 5: "workspace too small", 6: "non-finite value on the device"}
+          4: "unsupported shape", 5: "workspace too small", 6: "non-finite value on the device",
+          7: "index outside its buffer (debug build)"}
 
 
 class WildcatError(RuntimeError):
@@ -46,6 +47,17 @@ EXPORTS = [
 ]
 
 _lib = None
+
+
+def use_debug_library(debug: bool = True) -> None:
+    """Switch to the bounds-checked build (libwildcat_debug.so, built by
+    `python -m coreset_attention_approximation_b200.build --debug`): its kernels
+    check every data-dependent index (pivots, ranks) against its buffer and
+    record WC_ERR_BOUNDS instead of making the access.  Takes effect for calls
+    made after it."""
+    global LIB_PATH, _lib
+    LIB_PATH = os.path.join(HERE, "libwildcat_debug.so" if debug else "libwildcat.so")
+    _lib = None
 
 
 def lib():

@@ -86,7 +86,10 @@ typedef enum {
     WC_ERR_TIMEOUT = 3,      /* a device-side wait ran out (recorded on the device) */
     WC_ERR_UNSUPPORTED = 4,  /* valid but not implemented (e.g. d not in {64, 128} on a path) */
     WC_ERR_WORKSPACE = 5,    /* ws_bytes < wc_workspace_bytes(shape) */
-    WC_ERR_NUMERIC = 6       /* non-finite value met on the device */
+    WC_ERR_NUMERIC = 6,      /* non-finite value met on the device */
+    WC_ERR_BOUNDS = 7        /* an index outside its buffer (pivot, rank), recorded by the
+                                bounds-checked debug build (libwildcat_debug.so), which
+                                skips the access instead of faulting */
 } wc_status;
 
 typedef enum { WC_F32 = 0, WC_BF16 = 1 } wc_dtype;

@@ -47,9 +47,25 @@ def test_library_exports_every_declared_function(lib):
     assert set(wildcat.EXPORTS) <= exported
 
 
+def test_debug_library_exports_the_same_functions(lib):
+    """The bounds-checked build (libwildcat_debug.so) is the same ABI."""
+    path = os.path.join(os.path.dirname(wildcat.LIB_PATH), "libwildcat_debug.so")
+    if not os.path.exists(path):
+        from coreset_attention_approximation_b200 import build
+
+        build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (wc_\w+)$", out, flags=re.M))
+    assert not [n for n in declared_functions() if n not in exported]
+    d = ctypes.CDLL(path)
+    d.wc_status_string.restype = ctypes.c_char_p
+    assert d.wc_status_string(7) == b"index outside its buffer (debug build)"
+
+
 def test_status_strings(lib):
     assert lib.wc_status_string(0) == b"ok"
     assert lib.wc_status_string(5) == b"workspace too small"
+    assert lib.wc_status_string(7) == b"index outside its buffer (debug build)"
     assert lib.wc_status_string(99) == b"unknown status"
 
 
