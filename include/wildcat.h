@@ -26,8 +26,11 @@
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *     call is asynchronous on it; argument errors are returned before any
  *     launch, launch errors as WC_ERR_CUDA.  Errors that a kernel meets on
- *     the device (a wait that ran out, a non-finite factor) are recorded in
- *     the workspace and reported by wc_check_device_status.
+ *     the device (a wait that ran out, a non-finite factor, and in the
+ *     bounds-checked build libwildcat_debug.so an index outside its buffer)
+ *     are recorded in the workspace and reported by wc_check_device_status.
+ *   - No call allocates or synchronises (wc_check_device_status aside), so
+ *     select, weights, attend and forward can be captured into a CUDA graph.
  *   - Tensors are dense, row-major, 16-byte aligned:
  *       Q   [B, Hq,  n_q, d]    dtype
  *       K   [B, Hkv, n_k, d]    dtype
