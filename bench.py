@@ -38,9 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # dram bytes (read + write) per select launch per unit, from a one-pass ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current select
-# kernel on the named workload: long = 9.305450 TB + 8.889099 GB over 8 units
+# kernel on the named workload: long = 9.306759 TB + 8.881209 GB over 8 units
 # (profiles/select_rpcholesky_long8.md).  Other workloads: not captured.
-SELECT_DRAM_BYTES_PER_UNIT = {"long": (9.305450e12 + 8.889099e9) / 8}
+SELECT_DRAM_BYTES_PER_UNIT = {"long": (9.306759e12 + 8.881209e9) / 8}
 
 
 def load_peaks():
