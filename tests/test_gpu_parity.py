@@ -316,3 +316,23 @@ def test_forward_graph_replays_match_eager(kw):
         ref = run_gpu(Qh, Kh, Vh, w.r, seed=3, **kw)
         for k in ("out", "piv", "rank", "F", "W"):
             assert torch.equal(o[k].cpu(), ref[k]), k
+
+
+@pytest.mark.parametrize("d,deficient", [(128, False), (64, False), (128, True)])
+def test_attention_many_query_tiles(d, deficient):
+    """Attention over 40 ragged query tiles x 8 heads (no key split); r = 640
+    gives an odd number of key tiles (5); with `deficient` the second kv head's
+    keys have 6 distinct rows, so its query tiles see one key tile while the
+    first head's see five."""
+    w = WORKLOADS["long"].replace(hq=8, hkv=2, n_k=4096, n_q=5000, r=640, d=d)
+    Q, K, V = make_inputs(w, seed=51)
+    if deficient:
+        g = torch.Generator().manual_seed(51)
+        base = torch.randn(6, d, generator=g, dtype=torch.float64) * 0.3
+        idx = torch.randint(0, 6, (w.n_k,), generator=g)
+        idx[:6] = torch.arange(6)
+        K[0, 1] = base[idx].to(K.dtype)
+    rep = compare(Q, K, V, w.r, seed=51, tol_w=2e-3)
+    if deficient:
+        res = run_gpu(Q, K, V, w.r, seed=51)
+        assert int(res["rank"][0, 1]) == 6 and int(res["rank"][0, 0]) == w.r, rep
