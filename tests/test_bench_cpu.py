@@ -1,0 +1,41 @@
+"""bench.py on the CPU: the reference arm's JSON line (the oracle timed on the
+host) and the algorithmic byte and flop counts the roofline divides by."""
+
+import json
+import os
+import subprocess
+import sys
+
+import bench
+from coreset_attention_approximation_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_counts_of_the_long_workload():
+    w = WORKLOADS["long"]
+    # per unit and step j: K read (n d 2), factor prefix read (4 n j), column written (4 n)
+    n, r, d = w.n_k, w.r, w.d
+    per_unit = sum(n * d * 2 + 4 * n * j + 4 * n for j in range(r))
+    assert bench.select_bytes(w) == per_unit * w.hkv == 9350143803392
+    f1, f2 = bench.gemm_flops(w)
+    assert f1 == f2 == 2 * r * n * (d + w.dv + 1) * w.hkv
+    # bins: each of B bins selects r / B pivots over n / B keys
+    assert bench.select_bytes(w, bins=8) == 8 * w.hkv * sum((n // 8) * d * 2 + 4 * (n // 8) * (j + 1)
+                                                            for j in range(r // 8))
+    # centred keys stream as fp32
+    assert bench.select_bytes(w, center=True) - bench.select_bytes(w) == n * r * d * 2 * w.hkv
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "3", "--ref-pivots", "32"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT, check=True).stdout
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["config"]["workload"] == "tiny" and d["dtype"] == "f64"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
