@@ -291,7 +291,15 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
     if ((tid & 31) == 0 && lmax > 0.0) atomicMax(&us->hmax_bits, (unsigned long long)__double_as_longlong(lmax));
-    bool alive = unit_barrier(&us->bar, a.C, 1, a.timeout_ns, status, &bc.ok);
+    // the unit's blocks meet; a unit of one block only needs its own threads
+    auto unit_sync = [&](uint32_t epoch) -> bool {
+        if (a.C == 1) {
+            __syncthreads();
+            return true;
+        }
+        return unit_barrier(&us->bar, a.C, epoch, a.timeout_ns, status, &bc.ok);
+    };
+    bool alive = unit_sync(1);
     // The factor is taken of the shifted kernel H' = exp(beta K K^T - M): every
     // entry is at most 1 (Cauchy-Schwarz), the diagonal's maximum is 1, and the
     // pivots, the stop rule (relative to the diagonal's maximum) and the weights
@@ -314,7 +322,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
         const double tot = block_scan<NT>(sum, scan);
         if (tid == 0) part[blk] = tot;
     }
-    if (alive) alive = unit_barrier(&us->bar, a.C, 2, a.timeout_ns, status, &bc.ok);
+    if (alive) alive = unit_sync(2);
     const double hmax = 1.0;  // the shifted diagonal's maximum
 
     int final_rank = alive ? r : 0;
@@ -382,8 +390,10 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
                 us->d_s = ds;
                 us->stop = stop;
                 if (!stop) a.piv[(size_t)unit * r + j] = r0 + sl + (unit % a.bins) * a.bin_keys;
-                __threadfence();
-                st_release_u32(&us->pivflag, (uint32_t)j + 1u);
+                if (a.C > 1) {  // the unit's other blocks wait for it
+                    __threadfence();
+                    st_release_u32(&us->pivflag, (uint32_t)j + 1u);
+                }
                 bc.s = r0 + sl;
                 bc.d_s = ds;
                 bc.stop = stop;
@@ -466,7 +476,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
             const double tot = block_scan<NT>(sum, scan);
             if (tid == 0) part[(size_t)((j + 1) & 1) * kMaxBlocksPerUnit + blk] = tot;
         }
-        if (!unit_barrier(&us->bar, a.C, (uint32_t)j + 3u, a.timeout_ns, status, &bc.ok)) {
+        if (!unit_sync((uint32_t)j + 3u)) {
             final_rank = j + 1;
             alive = false;
             break;
