@@ -332,6 +332,7 @@ def run_ours(args, world, rank, local):
     del pipe
 
     kernels = kernel_breakdown(step)
+    approx = approximation_error(Q, K, V, out, w, args.bins)
 
     def gemm_steps():
         # weights and attention back to back, without the select before them
@@ -386,6 +387,7 @@ def run_ours(args, world, rank, local):
         "compress_attend_tokens_per_s": tokens / ((sel_avg + wts_avg + att_avg) * 1e-3),
         "gemm": gemm_report(kernels, f1, f2, peaks),
         "gemm_alone": gemm_alone_report(alone, f1, f2, peaks),
+        "approximation": approx,
         "kernels_ms": kernels,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -447,6 +449,30 @@ def gemm_report(kernels, f1, f2, peaks):
             tf = flops / (ms * 1e-3) / 1e12
             rep[name] = {"ms": ms, "tflops": tf, "frac": tf / sustained, "frac_burst": tf / burst, "flops": flops}
     return rep
+
+
+def approximation_error(Q, K, V, out, w, bins, nq_s=4096, max_heads=16):
+    """How far the coreset attention is from exact softmax attention (for
+    reporting only, outside the timed region): exact attention in fp32 with
+    plain torch matmuls on a seeded subsample of at most `nq_s` queries per head
+    (the first `max_heads` query heads), against the path's output rows.
+    ||out - exact||_F / ||exact||_F per head."""
+    beta = 1.0 / math.sqrt(w.d)
+    g = torch.Generator().manual_seed(0)
+    idx = torch.randperm(w.n_q, generator=g)[:min(nq_s, w.n_q)].to(Q.device)
+    group = w.hq // w.hkv
+    errs = []
+    with torch.no_grad():
+        for z in range(min(w.batch * w.hq, max_heads)):
+            b, h = divmod(z, w.hq)
+            q = Q[b, h, idx].float()
+            k, v = K[b, h // group].float(), V[b, h // group].float()
+            exact = torch.cat([torch.softmax((q[i:i + 512] @ k.T) * beta, dim=-1) @ v
+                               for i in range(0, q.shape[0], 512)])
+            errs.append(float((out[b, h, idx] - exact).norm() / exact.norm()))
+    return {"kind": "||out - exact||_F / ||exact||_F per head, exact softmax attention in fp32",
+            "queries_per_head": int(idx.numel()), "heads": len(errs), "bins": bins,
+            "rel_err_mean": statistics.mean(errs), "rel_err_max": max(errs)}
 
 
 def gemm_alone_report(kernels, f1, f2, peaks):

@@ -39,3 +39,23 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_approximation_error_of_exact_attention_is_zero():
+    """The bench's accuracy report measures against exact softmax attention:
+    handed the oracle's exact attention it reports (almost) zero, handed the
+    coreset attention of a small coreset a clearly positive error."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from coreset_attention_approximation_b200.workloads import make_inputs
+
+    w = WORKLOADS["tiny"].replace(n_k=256, n_q=64, r=8)
+    Q, K, V = make_inputs(w, seed=3)
+    beta = 1.0 / np.sqrt(w.d)
+    exact = torch.from_numpy(oracle.exact_attention(Q[0, 0], K[0, 0], V[0, 0], beta))[None, None].float()
+    rep = bench.approximation_error(Q, K, V, exact, w, 1)
+    assert rep["queries_per_head"] == 64 and rep["heads"] == 1 and rep["rel_err_max"] < 1e-5
+    approx = torch.from_numpy(oracle.forward(Q, K, V, w.r, seed=0)["out"]).float()
+    assert bench.approximation_error(Q, K, V, approx, w, 1)["rel_err_max"] > 1e-3
