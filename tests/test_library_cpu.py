@@ -113,3 +113,39 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "wc_oracle" not in text, f
+
+
+def test_every_entry_point_checks_its_arguments(lib):
+    """weights, attend, forward and the allocation-free attend refuse null and
+    misaligned pointers, short workspaces and invalid shapes before any
+    launch, so no GPU is needed to see the codes."""
+    s = wildcat.make_shape(1, 2, 1, 512, 16, 64, 64, 32, torch.bfloat16)
+    ok = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    big = 1 << 30
+    # weights: K, V, piv, F, rank, Ks, W
+    assert lib.wc_weights(ctypes.byref(s), None, ok, ok, ok, ok, ok, ok, ok, big, None) == 1
+    assert lib.wc_weights(ctypes.byref(s), ok, ok, ok, ok, ok, ok, mis, ok, big, None) == 1
+    assert lib.wc_weights(ctypes.byref(s), ok, ok, ok, ok, ok, ok, ok, ok, 1024, None) == 5
+    # attend: Q, Ks, W, rank, out
+    assert lib.wc_attend(ctypes.byref(s), None, ok, ok, ok, ok, ok, big, None) == 1
+    assert lib.wc_attend(ctypes.byref(s), ok, ok, ok, ok, mis, ok, big, None) == 1
+    assert lib.wc_attend(ctypes.byref(s), ok, ok, ok, ok, ok, ok, 1024, None) == 5
+    # forward: Q, K, V, out, piv, rank, F, Ks, W (the last five nullable, then the workspace must hold them)
+    assert lib.wc_forward(ctypes.byref(s), ok, None, ok, ok, None, None, None, None, None, ok, big, None) == 1
+    assert lib.wc_forward(ctypes.byref(s), ok, ok, ok, ok, None, None, None, None, None, ok,
+                          wildcat.workspace_bytes(s), None) == 5
+    # allocation-free attend
+    assert lib.wc_attend_noalloc(ctypes.byref(s), None, ok, ok, ok, ok, None) == 1
+    # an invalid shape is refused by every call
+    bad = wildcat.make_shape(1, 3, 2, 512, 16, 64, 64, 32, torch.bfloat16)   # hq not a multiple of hkv
+    assert lib.wc_weights(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, ok, big, None) == 1
+    assert lib.wc_attend(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, big, None) == 1
+    assert lib.wc_forward(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, ok, ok, ok, big, None) == 1
+    assert lib.wc_attend_noalloc(ctypes.byref(bad), ok, ok, ok, ok, ok, None) == 1
+    # bins and centring: n and r must be multiples of bins; center is 0 or 1
+    for field, value in (("bins", 3), ("bins", -1), ("center", 2)):
+        b2 = wildcat.make_shape(1, 2, 1, 512, 16, 64, 64, 32, torch.bfloat16)
+        setattr(b2, field, value)
+        assert wildcat.workspace_bytes(b2) == 0
+        assert lib.wc_select(ctypes.byref(b2), ok, ok, ok, ok, ok, big, None) == 1
