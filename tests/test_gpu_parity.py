@@ -220,11 +220,19 @@ def test_running_max_rescale_large_dynamic_range():
     assert int(res["piv"][0, 0, 0]) == 500 and int(res["rank"][0, 0]) == 48
 
 
-@pytest.mark.parametrize("d,dv", [(32, 96), (128, 64), (64, 128)])
+@pytest.mark.parametrize("d,dv", [(32, 96), (128, 64), (64, 128), (256, 256), (8, 8), (256, 8)])
 def test_other_head_widths_bf16(d, dv):
-    # (32, 96) runs on CUDA cores, the others on the tensor-core kernel
+    # (128, 64) and (64, 128) run on the tensor-core kernel, the others on CUDA cores;
+    # 8 and 256 are the narrowest and widest heads the library takes
     w = WORKLOADS["vit"].replace(batch=1, hq=4, hkv=2, n_k=1500, n_q=300, d=d, dv=dv, r=100)
     compare(*make_inputs(w, seed=d + dv), w.r, seed=3)
+
+
+@pytest.mark.parametrize("d,dv", [(256, 256), (8, 8)])
+def test_extreme_head_widths_fp32(d, dv):
+    w = WORKLOADS["tiny"].replace(batch=1, hq=2, hkv=2, n_k=700, n_q=90, d=d, dv=dv, r=40)
+    rep = compare(*make_inputs(w, seed=d + 7), w.r, seed=5, tol_w=1e-5)
+    assert rep["err_out"] <= 1e-5
 
 
 def test_large_key_norms_factor_stays_finite():
