@@ -221,19 +221,6 @@ def forward(Q, K, V, r, seed=0, *, ws=None, stream=None, outputs=None, **kw):
     return o
 
 
-def forward_host(Q, K, V, r, seed=0, *, device="cuda", ws=None, stream=None, **kw):
-    """Host-buffer entry: copies Q, K, V (pinned CPU tensors) to the device,
-    runs forward, copies `out` back.  Returns the CPU output tensor."""
-    dq = Q.to(device, non_blocking=True)
-    dk = K.to(device, non_blocking=True)
-    dv = V.to(device, non_blocking=True)
-    res = forward(dq, dk, dv, r, seed, ws=ws, stream=stream, **kw)
-    out = torch.empty(res["out"].shape, dtype=torch.float32, pin_memory=True)
-    out.copy_(res["out"], non_blocking=True)
-    torch.cuda.current_stream().synchronize()
-    return out
-
-
 class ForwardGraph:
     """wc_forward captured once into a CUDA graph, then replayed: repeated
     forward passes over the same device buffers cost one graph launch instead
