@@ -144,6 +144,21 @@ def test_separate_calls_match_forward():
     assert torch.equal(full["W"], wts["W"]) and torch.equal(full["out"], out)
 
 
+def test_one_workspace_serves_the_three_calls():
+    """The README's step-by-step use: a workspace sized for the whole problem
+    is handed to select, weights and attend (attention with few queries, so
+    the split attention's rows live in it too)."""
+    w = WORKLOADS["kv"].replace(hq=8, hkv=2, n_k=4096, r=512, n_q=200)
+    Q, K, V = [t.cuda() for t in make_inputs(w, seed=12)]
+    full = wildcat.forward(Q, K, V, w.r, seed=12)
+    ws = wildcat.workspace(wildcat.shape_of(Q, K, V, w.r), K.device)
+    sel = wildcat.select(K, w.r, seed=12, ws=ws)
+    wts = wildcat.weights(K, V, sel["piv"], sel["F"], sel["rank"], w.r, ws=ws, seed=12)
+    out = wildcat.attend(Q, wts["Ks"], wts["W"], sel["rank"], w.n_k, ws=ws)
+    assert wildcat.check_device_status(ws) == 0
+    assert torch.equal(full["piv"], sel["piv"]) and torch.equal(full["W"], wts["W"]) and torch.equal(full["out"], out)
+
+
 def test_wait_timeout_is_reported_and_context_survives():
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     assert wildcat.selftest_wait_timeout(ws, 200) == 0
