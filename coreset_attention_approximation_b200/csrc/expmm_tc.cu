@@ -9,7 +9,11 @@
 //   l += sum_b P w_b             fp32, in the softmax warps
 // C = fp16 values (V, or the weights W scaled per column); w = 1 or the
 // normaliser column W[:, dv].  Weights: the (O, l, m) of each key split are
-// written for the solve; attention: out = O sigma / l.
+// written for the solve (with centred keys a per-key logit bias is added to S);
+// attention: out = O sigma / l, or, when the query tiles are too few to fill
+// the GPU, (O sigma, l, m) per split of the coreset, combined by
+// attend_combine_kernel.  The weight preparation (fp16 W, sigma, w) runs as
+// clusters of 8 blocks whose column maxima meet in distributed shared memory.
 //
 // Warp roles (384 threads): warp 0 loads A once and then the key tiles, warp 1
 // the value tiles (TMA, 3-stage rings); warp 2 owns TMEM and issues S = A B^T,
