@@ -1,8 +1,8 @@
 // wc_common.cuh — device helpers shared by the WildCat kernels (sm_100a).
 //
-// Status word, bounded waits, the Philox4x32-10 counter generator (Salmon,
-// Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC'11),
-// element loads and the workspace layout.
+// Status word, the debug build's bounds checks, bounded waits, the
+// Philox4x32-10 counter generator (Salmon, Moraes, Dror, Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC'11) and element loads.
 #pragma once
 
 #include <cuda_bf16.h>
