@@ -37,7 +37,7 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->ldf = f_ld(s.n_k);
     o->units = s.batch * s.hkv;
     o->esize = s.dtype == WC_BF16 ? 2 : 4;
-    o->nsplit = (s.n_k + kSplitKeys - 1) / kSplitKeys;
+    o->nsplit = (s.n_k + split_keys(s.n_k, o->units, s.r) - 1) / split_keys(s.n_k, o->units, s.r);
     o->r_pad = (s.r + 63) / 64 * 64;
     if (s.bins < 0 || (s.center != 0 && s.center != 1)) return WC_ERR_INVALID;
     o->bins = s.bins > 1 ? s.bins : 1;
@@ -58,7 +58,7 @@ Shape bin_view(const Shape& s) {
     b.n = s.n_all / s.bins;
     b.r = s.r_all / s.bins;
     b.ldf = f_ld(b.n);
-    b.nsplit = (b.n + kSplitKeys - 1) / kSplitKeys;
+    b.nsplit = (b.n + split_keys(b.n, b.units, b.r) - 1) / split_keys(b.n, b.units, b.r);
     b.r_pad = (b.r + 63) / 64 * 64;
     return b;
 }
@@ -77,7 +77,8 @@ WsLayout make_layout(const Shape& s) {
     const size_t U = (size_t)s.units_all, B = (size_t)s.bins;
     const size_t n = (size_t)s.n_all, r = (size_t)s.r_all, nb = n / B, rb = r / B;
     const size_t ldb = (size_t)f_ld((int32_t)nb);
-    const size_t nsb = (nb + kSplitKeys - 1) / kSplitKeys;
+    const int skb = split_keys((int)nb, (int)(U * B), (int)rb);
+    const size_t nsb = (nb + skb - 1) / skb;
     const size_t r_pad = (r + 63) / 64 * 64;
     const size_t kt_unit = U * s.d * (size_t)f_ld((int32_t)n), kt_bin = U * B * s.d * ldb;
     L.status = take(256);

@@ -763,7 +763,7 @@ wc_status launch_coreset_values_tc(const Shape& s, const void* Ks, const void* K
     a.a_head_rows = s.r;
     a.b_rows = s.n;
     a.nsplit = s.nsplit;
-    a.split_len = kSplitKeys;
+    a.split_len = split_keys(s.n, s.units, s.r);
     a.r = s.r;
     a.r_pad = s.r_pad;
     a.hq = s.hkv;

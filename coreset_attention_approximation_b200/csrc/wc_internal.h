@@ -11,7 +11,19 @@
 namespace wc {
 
 constexpr int kMaxBlocksPerUnit = 512;   // select: thread blocks that share one unit
-constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1
+constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1 (at most)
+// Keys per partial sum of C1 for units of n keys and r coreset rows:
+// kSplitKeys; or, for heads of at most kSplitKeys keys whose row tiles leave
+// SMs idle, up to 4 splits of whole 128-key tiles (so a few short heads still
+// spread over the GPU, while many short heads keep one block each).
+inline int split_keys(int n, int units, int r) {
+    if (n > kSplitKeys) return kSplitKeys;
+    const long tiles = (long)units * ((r + 127) / 128);
+    int want = tiles >= 148 ? 1 : (int)((148 + tiles - 1) / tiles);
+    if (want > 4) want = 4;
+    const int q = ((n + want - 1) / want + 127) / 128 * 128;
+    return q < 128 ? 128 : q;
+}
 constexpr int kCenterChunk = 1024;       // centring: keys per partial column sum
 constexpr int kAttendFill = 148;         // attention: blocks resident at once (one per SM of a B200)
 // Row of a C1 partial sum: O[0 .. dv), l, m, two unused floats (rows 16-byte aligned).

@@ -278,7 +278,7 @@ wc_status launch_coreset_values(const Shape& s, const void* Ks, const void* K, c
     e.status = reinterpret_cast<int*>(ws + L.status);
     e.out = ws + L.c1part;
     e.d = s.d; e.dv = s.dv; e.r = s.r;
-    e.nsplit = s.nsplit; e.split_len = kSplitKeys;
+    e.nsplit = s.nsplit; e.split_len = split_keys(s.n, s.units, s.r);
     e.beta = (float)s.beta;
     e.group = 1; e.hq = s.hkv;
     e.mode = kExpmmPartial;
