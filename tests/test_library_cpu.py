@@ -149,3 +149,22 @@ def test_every_entry_point_checks_its_arguments(lib):
         setattr(b2, field, value)
         assert wildcat.workspace_bytes(b2) == 0
         assert lib.wc_select(ctypes.byref(b2), ok, ok, ok, ok, ok, big, None) == 1
+
+
+def test_one_workspace_holds_every_calls_scratch(lib):
+    """A workspace sized for the whole problem (queries and values included)
+    holds the scratch of select (no queries, the binding's 8-wide placeholder
+    values), weights (no queries) and attend, with and without bins, centring
+    and the decode-sized attention split."""
+    cases = [
+        (1, 8, 8, 131072, 131072, 128, 128, 2048, {}),
+        (1, 32, 8, 32768, 256, 128, 128, 1024, {}),            # decode-sized: attention splits
+        (2, 16, 16, 4096, 4096, 64, 64, 256, {"center": True}),
+        (1, 8, 8, 131072, 131072, 128, 128, 2048, {"bins": 8}),
+        (1, 1, 1, 512, 512, 64, 64, 32, {}),
+    ]
+    for b, hq, hkv, n, nq, d, dv, r, kw in cases:
+        full = wildcat.workspace_bytes(wildcat.make_shape(b, hq, hkv, n, nq, d, dv, r, torch.bfloat16, **kw))
+        select = wildcat.workspace_bytes(wildcat.make_shape(b, hkv, hkv, n, 0, d, 8, r, torch.bfloat16, **kw))
+        weights = wildcat.workspace_bytes(wildcat.make_shape(b, hkv, hkv, n, 0, d, dv, r, torch.bfloat16, **kw))
+        assert 0 < select <= full and 0 < weights <= full, (n, r, kw)
