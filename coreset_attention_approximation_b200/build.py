@@ -18,7 +18,7 @@ LIB = os.path.join(HERE, "libwildcat.so")
 OBJDIR = os.path.join(HERE, "_build")
 SOURCES = ["api.cu", "select.cu", "weights.cu", "expmm_simt.cu", "expmm_tc.cu", "attend.cu", "noalloc.cu",
            "center.cu"]
-HEADERS = ["wc_common.cuh", "wc_internal.h", "wc_expmm.cuh", "wc_tc.cuh"]
+HEADERS = ["wc_common.cuh", "wc_internal.h", "wc_expmm.cuh", "wc_tc.cuh", "wc_exp2.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

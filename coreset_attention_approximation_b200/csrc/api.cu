@@ -38,7 +38,7 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->units = s.batch * s.hkv;
     o->esize = s.dtype == WC_BF16 ? 2 : 4;
     o->nsplit = (s.n_k + split_keys(s.n_k, o->units, s.r) - 1) / split_keys(s.n_k, o->units, s.r);
-    o->r_pad = (s.r + 63) / 64 * 64;
+    o->r_pad = (s.r + 127) / 128 * 128;
     if (s.bins < 0 || (s.center != 0 && s.center != 1)) return WC_ERR_INVALID;
     o->bins = s.bins > 1 ? s.bins : 1;
     if (s.n_k % o->bins || s.r % o->bins) return WC_ERR_INVALID;
@@ -59,7 +59,7 @@ Shape bin_view(const Shape& s) {
     b.r = s.r_all / s.bins;
     b.ldf = f_ld(b.n);
     b.nsplit = (b.n + split_keys(b.n, b.units, b.r) - 1) / split_keys(b.n, b.units, b.r);
-    b.r_pad = (b.r + 63) / 64 * 64;
+    b.r_pad = (b.r + 127) / 128 * 128;
     return b;
 }
 
@@ -79,7 +79,7 @@ WsLayout make_layout(const Shape& s) {
     const size_t ldb = (size_t)f_ld((int32_t)nb);
     const int skb = split_keys((int)nb, (int)(U * B), (int)rb);
     const size_t nsb = (nb + skb - 1) / skb;
-    const size_t r_pad = (r + 63) / 64 * 64;
+    const size_t r_pad = (r + 127) / 128 * 128;
     const size_t kt_unit = U * s.d * (size_t)f_ld((int32_t)n), kt_bin = U * B * s.d * ldb;
     L.status = take(256);
     L.sync = take(sizeof(UnitSync) * U * B);
@@ -235,6 +235,13 @@ wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_m
     if (timeout_ms == 0 || timeout_ms > 60000) return WC_ERR_INVALID;
     return launch_wait_selftest(static_cast<char*>(ws), (uint64_t)timeout_ms * 1000000ull,
                                 static_cast<cudaStream_t>(stream));
+}
+
+wc_status wc_selftest_exp2(const float* x, float* y, int64_t n, int32_t method, void* stream) {
+    if (n < 0 || (method != 0 && method != 1)) return WC_ERR_INVALID;
+    if (n == 0) return WC_OK;
+    if (!x || !y || ((uintptr_t)x & 3u) || ((uintptr_t)y & 3u)) return WC_ERR_INVALID;
+    return launch_exp2_selftest(x, y, n, method, static_cast<cudaStream_t>(stream));
 }
 
 const char* wc_status_string(wc_status status) {

@@ -35,6 +35,7 @@
 #include <cudaTypedefs.h>
 
 #include "wc_common.cuh"
+#include "wc_exp2.cuh"
 #include "wc_expmm.cuh"
 #include "wc_internal.h"
 #include "wc_tc.cuh"
@@ -62,6 +63,24 @@ static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "r
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;  // log2 units: P stays below 2^8 between rescales
 constexpr uint64_t kTcTimeoutNs = 4000000000ull;
+// Exponentials moved off the exponential unit: of each row's 128 key columns,
+// kFmaExpCols run as exp2_fma2 on the FMA / ALU pipes (wc_exp2.cuh), the rest
+// as ex2.approx on the exponential unit.  Placement: the row's last columns
+// (kFmaExpSpread = 0), which a warp computes after handing the reference to
+// its partner, so the partner's exponentials have the unit to themselves; or
+// the last kFmaExpCols / 4 columns of every 32-column quarter (1).
+#ifndef WC_EXP2_FMA_COLS
+#define WC_EXP2_FMA_COLS 32
+#endif
+#ifndef WC_EXP2_FMA_SPREAD
+#define WC_EXP2_FMA_SPREAD 0
+#endif
+constexpr int kFmaExpCols = WC_EXP2_FMA_COLS;
+constexpr int kFmaExpSpread = WC_EXP2_FMA_SPREAD;
+static_assert(kFmaExpCols % 8 == 0 && kFmaExpCols >= 0 && kFmaExpCols <= BN, "whole column pairs per quarter");
+__host__ __device__ constexpr bool fma_exp_col(int col) {
+    return kFmaExpSpread ? (col % 32) >= 32 - kFmaExpCols / 4 : col >= BN - kFmaExpCols;
+}
 
 struct TcArgs {
     const int32_t* rank;
@@ -346,10 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < BN; j += 4) {
                         const float4 f = lds_f4_ordered(bv + j);
-                        sv[j] = fmaf(sv[j], cb, f.x);
-                        sv[j + 1] = fmaf(sv[j + 1], cb, f.y);
-                        sv[j + 2] = fmaf(sv[j + 2], cb, f.z);
-                        sv[j + 3] = fmaf(sv[j + 3], cb, f.w);
+                        const float2 lo = fma2(make_float2(sv[j], sv[j + 1]), make_float2(cb, cb), make_float2(f.x, f.y));
+                        const float2 hi =
+                            fma2(make_float2(sv[j + 2], sv[j + 3]), make_float2(cb, cb), make_float2(f.z, f.w));
+                        sv[j] = lo.x;
+                        sv[j + 1] = lo.y;
+                        sv[j + 2] = hi.x;
+                        sv[j + 3] = hi.y;
                     }
                 }
                 if (valid < BN) {
@@ -361,9 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) mq[i] = sv[i];
 #pragma unroll
-                for (int j = 8; j < BN; ++j) mq[j & 7] = fmaxf(mq[j & 7], sv[j]);
-                mt = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
-                           fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
+                for (int j = 8; j < BN; j += 2) mq[(j >> 1) & 7] = fmax3(mq[(j >> 1) & 7], sv[j], sv[j + 1]);
+                mt = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
                 if (MODE != kModeBias) mt *= cb;
             }
             // the reference after tile t - 1 (decided by the partner)
@@ -393,7 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // pass 2: P = 2^(S cb - mO) as fp16 pairs over the first 64 columns
                 const float* wv = reinterpret_cast<const float*>(sm + L::Wv + (t % NC) * BN * 4);
                 const float nm = -mO;
-                float lp[4] = {0.f, 0.f, 0.f, 0.f};
+                const float2 nm2 = make_float2(nm, nm), cb2 = make_float2(cb, cb);
+                float2 lp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     if (h == 3) {
@@ -417,24 +440,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        float p0, p1;
-                        if (MODE == kModeBias) {
-                            p0 = ex2_ordered(sh[j] + nm);
-                            p1 = ex2_ordered(sh[j + 1] + nm);
+                        // logits of the pair in log2 units, shifted by the reference
+                        const float2 s2 = make_float2(sh[j], sh[j + 1]);
+                        const float2 x2 = MODE == kModeBias ? add2(s2, nm2) : fma2(s2, cb2, nm2);
+                        float2 p;
+                        if (fma_exp_col(32 * h + j)) {
+                            p = exp2_fma2(x2);
                         } else {
-                            p0 = ex2_ordered(fmaf(sh[j], cb, nm));
-                            p1 = ex2_ordered(fmaf(sh[j + 1], cb, nm));
+                            p.x = ex2_ordered(x2.x);
+                            p.y = ex2_ordered(x2.y);
                         }
                         if (kQueries)
-                            lp[(j >> 1) & 3] = fmaf(p1, w[j + 1], fmaf(p0, w[j], lp[(j >> 1) & 3]));
+                            lp[(j >> 1) & 3] = fma2(p, make_float2(w[j], w[j + 1]), lp[(j >> 1) & 3]);
                         else
-                            lp[(j >> 1) & 3] += p0 + p1;
-                        const __half2 hp = __floats2half2_rn(p0, p1);
+                            lp[(j >> 1) & 3] = add2(lp[(j >> 1) & 3], p);
+                        const __half2 hp = __floats2half2_rn(p.x, p.y);
                         packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
                     }
                     tmem_st16u(tS + 16 * h, packed);
                 }
-                l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+                const float2 l01 = add2(lp[0], lp[1]), l23 = add2(lp[2], lp[3]);
+                l += (l01.x + l01.y) + (l23.x + l23.y);
                 tmem_wait_st();
                 if (grow && t > 0) {
                     // O holds key blocks 0..t-1 in the old reference: once the last of them
@@ -597,6 +623,25 @@ __global__ void attend_combine_kernel(const float* __restrict__ part, float* __r
     for (int k = 0; k < DV / 32; ++k) o[lane + 32 * k] = acc[k] * inv;
 }
 
+// The exp-GEMM's two ways to compute 2^x, over an array (for tests):
+// method 0 = exp2_fma2 (FMA / ALU pipes), 1 = ex2.approx.ftz (exponential unit).
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n, int method) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x * 2;
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 2; i < n; i += stride) {
+        const bool two = i + 1 < n;
+        const float a = x[i], b = two ? x[i + 1] : 0.f;
+        float2 v;
+        if (method == 0) {
+            v = exp2_fma2(make_float2(a, b));
+        } else {
+            v.x = ex2(a);
+            v.y = ex2(b);
+        }
+        y[i] = v.x;
+        if (two) y[i + 1] = v.y;
+    }
+}
+
 // V (bf16) -> fp16 copy for the value operand of the weights GEMM.
 __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, size_t count) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
@@ -718,6 +763,13 @@ wc_status launch_tc(int d, int dv, const CUtensorMap& A, const CUtensorMap& B, c
 }
 
 }  // namespace
+
+wc_status launch_exp2_selftest(const float* x, float* y, int64_t n, int method, cudaStream_t st) {
+    const int64_t pairs = (n + 1) / 2;
+    const int blocks = (int)(pairs < 256 * 1184 ? (pairs + 255) / 256 : 1184);
+    exp2_selftest_kernel<<<blocks, 256, 0, st>>>(x, y, n, method);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
 
 int attend_splits(const Shape& s) {
     // the attention's query tiles alone fill the GPU: no split

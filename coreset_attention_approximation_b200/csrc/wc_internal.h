@@ -54,7 +54,7 @@ struct WsLayout {
     size_t v16;       // half[units][n][dv]     values for the tensor-core weights GEMM
     size_t w16;       // half[units][r][dv]     column-scaled weights for attention
     size_t sigma;     // float[units][dv]       their column scales
-    size_t wn;        // float[units][r_pad]    normaliser column W[:, dv]
+    size_t wn;        // float[units][r_pad]    normaliser column W[:, dv], zero from rank to r_pad
     // centring (sizes 0 unless shape.center): per caller unit
     size_t kpart;     // double[units][n / kCenterChunk][d]  partial column sums
     size_t kbar;      // double[units][d]       mean key
@@ -79,7 +79,7 @@ struct Shape {
     int32_t units;         // batch * hkv
     int32_t esize;         // bytes per Q/K/V element
     int32_t nsplit;        // C1 partial sums
-    int32_t r_pad;         // r rounded up to 64
+    int32_t r_pad;         // r rounded up to 128 (whole key tiles of the attention's normaliser column)
     int32_t bins;          // key bins per unit (1: none); select and weights run on the bin view
     int32_t center;        // subtract each unit's mean key before the selection and the weights
     // the caller's problem, the same in the unit view and the bin view (sizes the workspace)
@@ -110,6 +110,8 @@ wc_status launch_key_shift(const Shape& s, const void* K, char* ws, cudaStream_t
 wc_status launch_attend(const Shape& s, const void* Q, const void* Ks, const float* W,
                         const int32_t* rank, float* out, char* ws, cudaStream_t st);
 wc_status launch_wait_selftest(char* ws, uint64_t timeout_ns, cudaStream_t st);
+// 2^x over an array: method 0 as the exp-GEMM's FMA-pipe polynomial, 1 on the exponential unit.
+wc_status launch_exp2_selftest(const float* x, float* y, int64_t n, int method, cudaStream_t st);
 
 // Tensor-core path (bf16 inputs, d and dv in {64, 128}).
 bool tc_supported(const Shape& s);

@@ -43,7 +43,7 @@ class WcShape(ctypes.Structure):
 EXPORTS = [
     "wc_f_ld", "wc_workspace_bytes", "wc_forward_workspace_bytes", "wc_select", "wc_weights", "wc_attend",
     "wc_forward", "wc_check_device_status", "wc_selftest_wait_timeout", "wc_status_string",
-    "wc_attend_noalloc",
+    "wc_attend_noalloc", "wc_selftest_exp2",
 ]
 
 _lib = None
@@ -83,6 +83,8 @@ def lib():
         L.wc_selftest_wait_timeout.restype = i32
         L.wc_status_string.argtypes, L.wc_status_string.restype = [i32], ctypes.c_char_p
         L.wc_attend_noalloc.argtypes, L.wc_attend_noalloc.restype = [sp, vp, vp, vp, vp, vp, vp], i32
+        L.wc_selftest_exp2.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int32, vp]
+        L.wc_selftest_exp2.restype = i32
         _lib = L
     return _lib
 
@@ -334,3 +336,11 @@ def check_device_status(ws, stream=None) -> int:
 
 def selftest_wait_timeout(ws, timeout_ms, stream=None) -> int:
     return int(lib().wc_selftest_wait_timeout(_ptr(ws), ws.numel(), timeout_ms, _stream(stream)))
+
+
+def selftest_exp2(x, method=0, stream=None):
+    """2^x for an fp32 CUDA tensor as the tensor-core kernels compute it:
+    method 0 on the FMA / ALU pipes (the polynomial), 1 on the exponential unit."""
+    y = torch.empty_like(x)
+    _check(lib().wc_selftest_exp2(_ptr(x), _ptr(y), x.numel(), method, _stream(stream)), "wc_selftest_exp2")
+    return y

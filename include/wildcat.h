@@ -196,6 +196,22 @@ wc_status wc_check_device_status(void* ws, void* stream);
 wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_ms, void* stream);
 
 /*
+ * Evaluates over x[0 .. n) (device memory, fp32) the two ways the tensor-core
+ * attention and weights kernels compute 2^x, writing y[0 .. n):
+ *   method 0  a polynomial on the FMA / ALU pipes: x = n + f with n = rint(x)
+ *             and f in [-1/2, 1/2] (additive range reduction after Cody and
+ *             Waite), 2^f by a degree-3 relative-minimax (Remez) polynomial,
+ *             2^n added to the exponent; relative error <= 2^-13.5 for
+ *             -125 <= x <= 127, about 2^-125 returned below -125
+ *   method 1  the exponential unit (ex2.approx.ftz.f32)
+ * The kernels run part of every row's exponentials with method 0 to relieve
+ * the exponential unit, which the tensor pipe otherwise waits for.  For
+ * tests; asynchronous on `stream`; WC_ERR_INVALID for n < 0, a null or
+ * misaligned pointer or another method.
+ */
+wc_status wc_selftest_exp2(const float* x, float* y, int64_t n, int32_t method, void* stream);
+
+/*
  * attend_noalloc — the same result as wc_attend, for callers that cannot
  * allocate device memory or pass a workspace (an allocator that must not be
  * re-entered, a process whose memory budget is fixed up front, a plugin that
@@ -203,19 +219,27 @@ wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_m
  * deployment variant of the attend step.
  *   - Scratch: a fixed 16 MiB array in device memory owned by the library
  *     (every GPU that loads the library holds it until the process exits).
- *     Shapes that need more (2 * units * r * dv + 4 * units * (dv + r rounded
- *     up to 64) bytes, plus alignment) are refused with WC_ERR_WORKSPACE
- *     before any launch.  bf16 inputs with d, dv in {64, 128} use it; other
- *     shapes run on the CUDA-core kernel, which needs no scratch.
+ *     bf16 inputs with d, dv in {64, 128} use it; other shapes run on the
+ *     CUDA-core kernel, which needs no scratch.  With units = batch * hkv and
+ *     up(x) = x rounded up to a multiple of 256, a shape needs
+ *         256 + up(2 * units * r * dv) + up(4 * units * dv)
+ *             + up(4 * units * (r rounded up to 128))        bytes,
+ *     and shapes that need more than 16 MiB (16777216 bytes) are refused with
+ *     WC_ERR_WORKSPACE before any launch.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept per device number, for
+ *     the device's primary context (the one the CUDA runtime uses); callers
+ *     that make their own driver-API contexts current are not served.
  *   - No cudaMalloc, cudaFree or other allocating call is made.
  *   - Every call shares the one array and leaves its contents behind; the
  *     call clears what it needs cleared.  Calls whose execution overlaps on
  *     the GPU (other streams, other threads) race on it: serialise them.
- *   - A device-side wait that runs out ends the kernel cleanly but is not
- *     reported here (use wc_attend with a workspace to read such errors).
+ *   - The kernels record device-side errors (a wait that ran out, and in the
+ *     bounds-checked build an index outside its buffer) in a status word at
+ *     the start of the array, which each call clears first; they need it to
+ *     wind down cleanly, and no call reports it (use wc_attend with a
+ *     workspace and wc_check_device_status to read such errors).
  */
 wc_status wc_attend_noalloc(const wc_shape* shape, const void* Q, const void* Ks, const float* W,
                             const int32_t* rank, float* out, void* stream);
