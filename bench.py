@@ -8,10 +8,18 @@ workload through the C ABI, inputs resident in HBM.  Default workload `long`:
 The inputs (K, V, Q: 805 MB) and the factor F (8.6 GB) are far larger than the
 126 MB L2, so no flush is needed between steps.
 
-With N > 1 (torchrun, one process per GPU) every rank runs its own copy of the
-workload (independent units, no collective on the data path: weak scaling);
-the step time is the max over ranks.  `--impl reference` times the CPU oracle
-on a bounded sample of the same workload (rank 0 only).
+With N > 1 (torchrun, one process per GPU) the (batch, kv head) units of one
+problem are split across the ranks, with no collective on the data path (the
+units are independent); the step time is the max over ranks:
+  --scaling weak    (default) the problem is N workloads stacked along the
+                    batch: rank k owns batch block k, drawn with its own seed,
+                    and passes unit_base = k * units so its units draw the
+                    Philox streams they draw in one call over the whole stack
+  --scaling strong  the workload's own units, contiguous blocks of
+                    [k U / N, (k + 1) U / N) per rank (U = batch * kv heads)
+`--gather` adds one all-gather of the outputs after the timed region (timed
+apart).  `--impl reference` times the CPU oracle on one whole unit of the same
+workload (rank 0 only).
 """
 
 from __future__ import annotations
@@ -26,6 +34,7 @@ import sys
 import tempfile
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -36,10 +45,9 @@ from coreset_attention_approximation_b200.workloads import WORKLOADS, make_input
 METRIC = "WildCat forward tokens/sec at 1 B200; select HBM GB/s and GEMM TC-util vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# dram bytes (read + write) per select launch per unit, from a one-pass ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current select
-# kernel on the named workload: long = 9.306759 TB + 8.881209 GB over 8 units
-# (profiles/select_rpcholesky_long8.md).  Other workloads: not captured.
+# DRAM bytes (read + write) of the select kernel per unit and launch, measured
+# with ncu's dram__bytes_read.sum + dram__bytes_write.sum on the named workload:
+# long = 9.306759 TB + 8.881209 GB over 8 units.  Other workloads: not captured.
 SELECT_DRAM_BYTES_PER_UNIT = {"long": (9.306759e12 + 8.881209e9) / 8}
 
 
@@ -177,63 +185,135 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 def shard_seed(seed: int, rank: int) -> int:
-    """Each rank draws its own independent copy of the workload."""
+    """Seed of batch block `rank` of the weak-scaling problem (block 0: `seed`)."""
     return seed + 1000003 * rank
 
 
-# ------------------------------------------------------------------ oracle sample
+def unit_range(units: int, world: int, rank: int) -> tuple[int, int]:
+    """Rank `rank`'s contiguous block of `units` units: [rank U / N, (rank + 1) U / N)."""
+    return rank * units // world, (rank + 1) * units // world
 
-def oracle_sample(w, r_s: int = 512, nq_s: int = 4096, bins: int = 1, center: bool = False):
-    """Time the CPU oracle on a bounded sample of workload `w` and scale it to
-    the whole workload.  Sample: unit 0, select steps 0..r_s-1 (the select's
-    cost is n * sum_j (d + j) multiply-adds, so its time scales by that count),
-    the weights on those r_s pivots (C1 dominates: linear in r) and attention
-    for nq_s queries of one head (linear in queries and in r).  With bins the
-    select and weights sample is bin 0 of unit 0 (n/B keys, r/B pivots), scaled
-    by units x B; attention still covers r coreset rows."""
-    import numpy as np
 
+def local_problem(w, seed: int, world: int, rank: int, scaling: str):
+    """This rank's share of the job: (Q, K, V host tensors, the workload those
+    tensors form, unit_base, query tokens of the whole job per step).
+
+    weak: the job is `world` copies of the workload stacked along the batch;
+    rank k holds copy k (seed shard_seed(seed, k)), whose units are units
+    k U .. (k + 1) U - 1 of the stack.  strong: the workload itself; rank k
+    holds units unit_range(U, world, k), each unit as a batch entry of one kv
+    head with its hq / hkv query heads."""
+    U = w.batch * w.hkv
+    if scaling == "weak" or world == 1:
+        Q, K, V = make_inputs(w, seed=shard_seed(seed, rank))
+        return Q, K, V, w, rank * U, world * w.batch * w.n_q
+    lo, hi = unit_range(U, world, rank)
+    if hi <= lo:
+        raise SystemExit(f"--scaling strong needs at least one unit per rank ({U} units, {world} ranks)")
+    group = w.hq // w.hkv
+    Q, K, V = make_inputs(w, seed=seed)
+    Qr = Q.reshape(U, group, w.n_q, w.d)[lo:hi].contiguous()
+    Kr = K.reshape(U, 1, w.n_k, w.d)[lo:hi].contiguous()
+    Vr = V.reshape(U, 1, w.n_k, w.dv)[lo:hi].contiguous()
+    return Qr, Kr, Vr, w.replace(batch=hi - lo, hq=group, hkv=1), lo, w.batch * w.n_q
+
+
+def gather_units(out_local, units: int, world: int, rank: int):
+    """The strong split's outputs ([units_k, hq / hkv, n_q, dv] per rank, rank
+    k holding unit_range(units, world, k)) assembled in unit order on every
+    rank with one all-gather of equal-size blocks (padded to the largest
+    share)."""
+    import torch.distributed as dist
+
+    per = max(unit_range(units, world, k)[1] - unit_range(units, world, k)[0] for k in range(world))
+    lo, hi = unit_range(units, world, rank)
+    buf = torch.zeros((per,) + tuple(out_local.shape[1:]), dtype=out_local.dtype, device=out_local.device)
+    buf[: hi - lo] = out_local
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf)
+    return torch.cat([parts[k][: unit_range(units, world, k)[1] - unit_range(units, world, k)[0]]
+                      for k in range(world)])
+
+
+def l2_note(w) -> str:
+    """Whether a step's working set (Q, K, V, the factor F and the output)
+    exceeds the 126 MB L2, so no flush is needed between steps."""
+    es = 2 if w.dtype == "bf16" else 4
+    units = w.batch * w.hkv
+    ldf = (w.n_k + 63) // 64 * 64
+    ws = (units * w.n_k * (w.d + w.dv) * es + w.batch * w.hq * w.n_q * (w.d * es + w.dv * 4)
+          + units * w.r * ldf * 4)
+    if ws > 126e6:
+        return f"working set {ws / 1e6:.0f} MB > 126 MB L2 (no flush)"
+    return f"working set {ws / 1e6:.0f} MB fits in the 126 MB L2 (no flush; L2-resident figures are context)"
+
+
+def job_config(w, args, world: int) -> dict:
+    """The `config` object of the JSON line, the same in both arms."""
+    return {
+        "workload": w.name, "batch": w.batch, "heads_q": w.hq, "heads_kv": w.hkv, "n_k": w.n_k,
+        "n_q": w.n_q, "d": w.d, "dv": w.dv, "r": w.r, "keys": w.keys, "seed": args.seed,
+        "bins": args.bins, "center": bool(args.center),
+        "l2": l2_note(w),
+        "parallelism": (f"{args.scaling} split of (batch, kv head) units over {world} ranks" if world > 1
+                        else "one GPU, all units"),
+    }
+
+
+# ------------------------------------------------------------------ oracle on one unit
+
+def oracle_unit(w, nq_s: int = 4096, bins: int = 1, center: bool = False, r_s: int | None = None):
+    """Time the CPU oracle on one whole (batch, kv head) unit of workload `w`:
+    unit 0's selection (every pivot step; with bins, every bin), its Nystrom
+    weights, and attention for min(nq_s, n_q) queries of one of its query heads
+    over its coreset (the union of the bins' coresets).  The workload's time is
+    units x (select + weights) + query heads x attention x n_q / sampled
+    queries: one multiplication by the unit count, and, when n_q > nq_s, the
+    attention scaled by the query count (it is linear in the queries).
+    r_s (tests only) cuts the selection to its first r_s steps per bin."""
     import oracle
 
     Q, K, V = make_inputs(w.replace(batch=1, hq=w.hq // w.hkv, hkv=1))
     beta = 1.0 / math.sqrt(w.d)
     nb, rb = w.n_k // bins, w.r // bins
-    r_s = min(r_s, rb)
+    steps = rb if r_s is None else min(r_s, rb)
     nq_s = min(nq_s, w.n_q)
     Kn, Vn = K[0, 0].double().numpy(), V[0, 0].double().numpy()
     if center:
         Kn = oracle.center_keys(Kn)
-    Kn, Vn = Kn[:nb], Vn[:nb]
-    t0 = time.perf_counter()
-    sel = oracle.rpcholesky(Kn, r_s, beta, seed=0, unit=0)
-    t1 = time.perf_counter()
-    k = sel["rank"]
-    Wt = oracle.nystrom_weights(Kn, Vn, sel["piv"], k, beta)
+    t_sel = t_w = 0.0
+    Ks_parts, W_parts = [], []
+    for b in range(bins):
+        Kb, Vb = Kn[b * nb:(b + 1) * nb], Vn[b * nb:(b + 1) * nb]
+        t0 = time.perf_counter()
+        sel = oracle.rpcholesky(Kb, steps, beta, seed=0, unit=b)
+        t1 = time.perf_counter()
+        k = sel["rank"]
+        if k > 0:
+            W_parts.append(oracle.nystrom_weights(Kb, Vb, sel["piv"], k, beta))
+            Ks_parts.append(Kb[sel["piv"][:k]])
+        t2 = time.perf_counter()
+        t_sel += t1 - t0
+        t_w += t2 - t1
     t2 = time.perf_counter()
-    oracle.coreset_attend(Q[0, 0, :nq_s].double().numpy(), Kn[sel["piv"][:k]], Wt, beta)
-    t3 = time.perf_counter()
-
-    def sel_work(r):
-        return nb * (r * w.d + r * (r - 1) / 2.0)
-
-    units = w.batch * w.hkv * bins
+    oracle.coreset_attend(Q[0, 0, :nq_s].double().numpy(), np.concatenate(Ks_parts), np.concatenate(W_parts), beta)
+    t_att = time.perf_counter() - t2
+    units = w.batch * w.hkv
     heads = w.batch * w.hq
-    t_sel = (t1 - t0) * sel_work(rb) / sel_work(r_s)
-    t_w = (t2 - t1) * rb / r_s
-    t_att = (t3 - t2) * (w.n_q / nq_s) * (w.r / r_s)
-    total = units * (t_sel + t_w) + heads * t_att
+    total = units * (t_sel + t_w) + heads * t_att * (w.n_q / nq_s)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cut = f" (selection cut to {steps} of {rb} steps per bin: not a timing of the workload)" if steps < rb else ""
     return {
         "value": w.batch * w.n_q / total,
         "unit": "tokens/s",
         "cores": cores,
         "kind": "oracle",
-        "sample": (f"{w.name}{f' bins={bins}' if bins > 1 else ''}{' centred' if center else ''}: "
-                   f"unit 0 of {units}; select steps 0..{r_s - 1} of {rb} "
-                   f"({t1 - t0:.1f} s, scaled by n*sum_j(d+j)); weights on {r_s} pivots ({t2 - t1:.1f} s, "
-                   f"scaled x r/{r_s}); attend {nq_s} queries ({t3 - t2:.1f} s, scaled x n_q/{nq_s} x r/{r_s}); "
-                   f"whole-workload estimate {total:.0f} s"),
-        "sample_seconds": t3 - t0,
+        "sample": (f"{w.name}{f' bins={bins}' if bins > 1 else ''}{' centred' if center else ''}: unit 0 in full "
+                   f"(select {t_sel:.1f} s, weights {t_w:.1f} s, attention {t_att:.2f} s for {nq_s} of {w.n_q} "
+                   f"queries of one head), x {units} units and x {heads} heads x {w.n_q}/{nq_s} for attention: "
+                   f"{total:.0f} s for the workload{cut}"),
+        "sample_seconds": t_sel + t_w + t_att,
+        "workload_seconds": total,
     }
 
 
@@ -242,12 +322,13 @@ def oracle_sample(w, r_s: int = 512, nq_s: int = 4096, bins: int = 1, center: bo
 def run_ours(args, world, rank, local):
     from coreset_attention_approximation_b200 import wildcat
 
-    w = WORKLOADS[args.workload]
+    wj = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    Qh, Kh, Vh = make_inputs(w, seed=shard_seed(args.seed, rank))
+    # this rank's units (w: the workload they form on this GPU)
+    Qh, Kh, Vh, w, unit_base, job_tokens = local_problem(wj, args.seed, world, rank, args.scaling)
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
-    shape = wildcat.shape_of(Q, K, V, w.r, seed=args.seed, bins=args.bins, center=args.center)
+    shape = wildcat.shape_of(Q, K, V, w.r, seed=args.seed, bins=args.bins, center=args.center, unit_base=unit_base)
     ws = wildcat.workspace(shape, dev)
     o = wildcat._outputs(shape, dev, K.dtype)
     out = torch.empty(w.batch, w.hq, w.n_q, w.dv, dtype=torch.float32, device=dev)
@@ -311,7 +392,7 @@ def run_ours(args, world, rank, local):
     h2d = Qp.numel() * Qp.element_size() + Kp.numel() * Kp.element_size() + Vp.numel() * Vp.element_size()
     d2h = outp[0].numel() * outp[0].element_size()
     pipe = wildcat.HostPipeline(Qp, Kp, Vp, w.r, seed=args.seed, device=dev, stream=stream, ws=ws, outputs=o,
-                                bins=args.bins, center=args.center)
+                                bins=args.bins, center=args.center, unit_base=unit_base)
 
     def batches(k):
         return [(Qp, Kp, Vp, outp[i % 2]) for i in range(k)]
@@ -353,7 +434,18 @@ def run_ours(args, world, rank, local):
     wts_avg, att_avg = sum(wts_ms) / len(wts_ms), sum(att_ms) / len(att_ms)
     captured = w.name in SELECT_DRAM_BYTES_PER_UNIT and args.bins == 1 and not args.center
     traffic = SELECT_DRAM_BYTES_PER_UNIT[w.name] * w.batch * w.hkv if captured else None
-    tokens = w.batch * w.n_q * world
+    tokens = job_tokens
+    gather = None
+    if args.gather and world > 1 and args.scaling == "strong":
+        # outputs of all ranks assembled in unit order on every rank (after the timed region)
+        barrier(world)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        full = gather_units(out.reshape(w.batch, w.hq, w.n_q, w.dv), wj.batch * wj.hkv, world, rank)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gather = {"ms": max_over_ranks(g0.elapsed_time(g1), world), "bytes_out": full.numel() * full.element_size(),
+                  "collective": "all_gather (NCCL)"}
     res = {
         "metric": METRIC,
         "value": tokens / (ms_step * 1e-3),
@@ -363,17 +455,11 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded generator; no dataset)",
-        "config": {
-            "workload": w.name, "batch": w.batch, "heads_q": w.hq, "heads_kv": w.hkv, "n_k": w.n_k,
-            "n_q": w.n_q, "d": w.d, "dv": w.dv, "r": w.r, "keys": w.keys, "seed": args.seed,
-            "bins": args.bins, "center": bool(args.center),
-            "l2": "inputs and factor larger than L2 (no flush)",
-            "parallelism": f"independent units per rank x{world}",
-        },
+        "config": job_config(wj, args, world),
         "roofline": {
             "bound": "hbm", "kernel": "rpcholesky_kernel (select)", "achieved": achieved,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
@@ -395,7 +481,10 @@ def run_ours(args, world, rank, local):
         # counted on the profiled step (the same launches as every timed step)
         "gpu_launches": kernels.pop("launches") * args.steps,
         "clocks": clocks.summary(),
+        "units_on_rank0": w.batch * w.hkv,
     }
+    if gather:
+        res["gather"] = gather
     return res
 
 
@@ -495,24 +584,32 @@ def gemm_alone_report(kernels, f1, f2, peaks):
 
 
 def run_reference(args, world, rank):
+    """The oracle as the reference arm: every timed step times one whole unit
+    of the workload (oracle_unit) and scales it by the unit count.  A whole
+    unit of the long workload takes about 40 s on 16 host cores, so the timed
+    steps stop once `--ref-budget-s` seconds are spent (at least one runs);
+    the warm-up steps run the selection's first pivots only."""
     w = WORKLOADS[args.workload]
     if rank != 0:
         return None
     for _ in range(args.warmup):
-        oracle_sample(w, r_s=64, nq_s=256, bins=args.bins, center=args.center)
-    vals = []
-    last = None
+        oracle_unit(w, nq_s=256, bins=args.bins, center=args.center, r_s=min(16, w.r // args.bins))
+    vals, last, spent = [], None, 0.0
     for _ in range(args.steps):
-        last = oracle_sample(w, r_s=args.ref_pivots, nq_s=4096, bins=args.bins, center=args.center)
+        t0 = time.perf_counter()
+        last = oracle_unit(w, bins=args.bins, center=args.center, r_s=args.ref_pivots)
         vals.append(last["value"])
+        dt = time.perf_counter() - t0
+        spent += dt
+        if spent + dt > args.ref_budget_s:   # the next whole unit would overrun the budget
+            break
     v = statistics.median(vals)
     return {
-        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": w.batch * w.n_q / v * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator; no dataset)",
-        "config": {"workload": w.name, "batch": w.batch, "heads_q": w.hq, "heads_kv": w.hkv, "n_k": w.n_k,
-                   "n_q": w.n_q, "d": w.d, "dv": w.dv, "r": w.r, "keys": w.keys, "seed": args.seed,
-                   "bins": args.bins, "center": bool(args.center)},
+        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": len(vals),
+        "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": w.batch * w.n_q / v * 1e3,
+        "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": job_config(w, args, world),
         "impl": "reference",
         "cpu_baseline": {k: last[k] for k in ("value", "unit", "cores", "kind", "sample")} | {"value": v},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -527,7 +624,14 @@ def main():
     ap.add_argument("--workload", default="long", choices=sorted(WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-pivots", type=int, default=512, help="select steps in the oracle sample")
+    ap.add_argument("--ref-pivots", type=int, default=None,
+                    help="(tests only) cut the oracle's selection to this many steps per bin")
+    ap.add_argument("--ref-budget-s", type=float, default=150.0,
+                    help="reference arm: stop timing whole units once this many seconds are spent")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="N > 1: weak = N stacked workloads, one per rank; strong = the workload's units split")
+    ap.add_argument("--gather", action="store_true",
+                    help="strong scaling: all-gather the outputs after the timed region (timed apart)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bins", type=int, default=1,
                     help="divide-and-conquer selection: B key bins per head (n and r multiples of B)")
@@ -544,8 +648,8 @@ def main():
         else:
             res = run_ours(args, world, rank, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
-                cb = oracle_sample(WORKLOADS[args.workload], r_s=args.ref_pivots, bins=args.bins,
-                                   center=args.center)
+                cb = oracle_unit(WORKLOADS[args.workload], r_s=args.ref_pivots, bins=args.bins,
+                                 center=args.center)
                 res["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)

@@ -43,6 +43,8 @@ wc_status make_shape(const wc_shape* in, Shape* o) {
     o->bins = s.bins > 1 ? s.bins : 1;
     if (s.n_k % o->bins || s.r % o->bins) return WC_ERR_INVALID;
     o->center = s.center;
+    if (s.unit_base < 0 || ((int64_t)s.unit_base + o->units) * o->bins > (int64_t)UINT32_MAX) return WC_ERR_INVALID;
+    o->unit_base = s.unit_base;
     o->units_all = o->units;
     o->n_all = s.n_k;
     o->r_all = s.r;

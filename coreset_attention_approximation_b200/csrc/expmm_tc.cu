@@ -65,19 +65,29 @@ constexpr float kRescale = 8.0f;  // log2 units: P stays below 2^8 between resca
 constexpr uint64_t kTcTimeoutNs = 4000000000ull;
 // Exponentials moved off the exponential unit: of each row's 128 key columns,
 // kFmaExpCols run as exp2_fma2 on the FMA / ALU pipes (wc_exp2.cuh), the rest
-// as ex2.approx on the exponential unit.  Placement: the row's last columns
-// (kFmaExpSpread = 0), which a warp computes after handing the reference to
-// its partner, so the partner's exponentials have the unit to themselves; or
-// the last kFmaExpCols / 4 columns of every 32-column quarter (1).
+// as ex2.approx on the exponential unit; placed at the row's last columns
+// (kFmaExpSpread = 0) or at the last kFmaExpCols / 4 columns of every
+// 32-column quarter (1).  Measured on the B200 with 0, 16, 32 and 48 columns
+// in both placements: no split was faster than none (each 128-key tile is
+// bound by shared-memory bandwidth, not by the exponential unit), so none is
+// the default.
 #ifndef WC_EXP2_FMA_COLS
-#define WC_EXP2_FMA_COLS 32
+#define WC_EXP2_FMA_COLS 0
 #endif
 #ifndef WC_EXP2_FMA_SPREAD
 #define WC_EXP2_FMA_SPREAD 0
 #endif
+// The quarter of a tile's row before whose exponentials a softmax warp hands
+// the reference to its partner; 0 (as soon as it is decided, so the two
+// warps' exponentials overlap) measured 2-6 % faster than the last quarter.
+#ifndef WC_HANDOFF_QUARTER
+#define WC_HANDOFF_QUARTER 0
+#endif
 constexpr int kFmaExpCols = WC_EXP2_FMA_COLS;
+constexpr int kHandQuarter = WC_HANDOFF_QUARTER;
 constexpr int kFmaExpSpread = WC_EXP2_FMA_SPREAD;
 static_assert(kFmaExpCols % 8 == 0 && kFmaExpCols >= 0 && kFmaExpCols <= BN, "whole column pairs per quarter");
+static_assert(kHandQuarter >= 0 && kHandQuarter <= 3, "hand-over quarter");
 __host__ __device__ constexpr bool fma_exp_col(int col) {
     return kFmaExpSpread ? (col % 32) >= 32 - kFmaExpCols / 4 : col >= BN - kFmaExpCols;
 }
@@ -417,21 +427,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float2 nm2 = make_float2(nm, nm), cb2 = make_float2(cb, cb);
                 float2 lp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                 make_float2(0.f, 0.f)};
+                // Software-pipelined by 32-column quarter: iteration h issues the
+                // exponentials of quarter h (results written over the logits) between
+                // the packing and normaliser sums of quarter h - 1, whose inputs are
+                // ready by then, so the warp's in-order issue does not wait on the
+                // exponential unit's latency, and stores quarter h - 1 as fp16 pairs.
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    if (h == 3) {
-                        // hand the reference on before the last quarter: the partner's
-                        // exponentials start as this warp's drain from the unit
+                for (int h = 0; h <= 4; ++h) {
+                    if (h == kHandQuarter) {
+                        // hand the reference on: the partner's exponentials may start
                         if (t + 1 < T) pair_arrive(id_out);
                         handed = true;
                     }
-                    const float* sh = sv + 32 * h;
                     uint32_t packed[16];
                     float w[kQueries ? 32 : 1];
-                    if (kQueries) {
+                    if (kQueries && h > 0) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
-                            const float4 f = lds_f4_ordered(wv + 32 * h + j);
+                            const float4 f = lds_f4_ordered(wv + 32 * (h - 1) + j);
                             w[j] = f.x;
                             w[j + 1] = f.y;
                             w[j + 2] = f.z;
@@ -440,24 +453,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        // logits of the pair in log2 units, shifted by the reference
-                        const float2 s2 = make_float2(sh[j], sh[j + 1]);
-                        const float2 x2 = MODE == kModeBias ? add2(s2, nm2) : fma2(s2, cb2, nm2);
-                        float2 p;
-                        if (fma_exp_col(32 * h + j)) {
-                            p = exp2_fma2(x2);
-                        } else {
-                            p.x = ex2_ordered(x2.x);
-                            p.y = ex2_ordered(x2.y);
+                        if (h < 4) {
+                            // logits of the pair in log2 units, shifted by the reference
+                            const int c = 32 * h + j;
+                            const float2 s2 = make_float2(sv[c], sv[c + 1]);
+                            const float2 x2 = MODE == kModeBias ? add2(s2, nm2) : fma2(s2, cb2, nm2);
+                            float2 p;
+                            if (fma_exp_col(c)) {
+                                p = exp2_fma2(x2);
+                            } else {
+                                p.x = ex2_ordered(x2.x);
+                                p.y = ex2_ordered(x2.y);
+                            }
+                            sv[c] = p.x;
+                            sv[c + 1] = p.y;
                         }
-                        if (kQueries)
-                            lp[(j >> 1) & 3] = fma2(p, make_float2(w[j], w[j + 1]), lp[(j >> 1) & 3]);
-                        else
-                            lp[(j >> 1) & 3] = add2(lp[(j >> 1) & 3], p);
-                        const __half2 hp = __floats2half2_rn(p.x, p.y);
-                        packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                        if (h > 0) {
+                            const int c = 32 * (h - 1) + j;
+                            const float2 p = make_float2(sv[c], sv[c + 1]);
+                            if (kQueries)
+                                lp[(j >> 1) & 3] = fma2(p, make_float2(w[j], w[j + 1]), lp[(j >> 1) & 3]);
+                            else
+                                lp[(j >> 1) & 3] = add2(lp[(j >> 1) & 3], p);
+                            packed[j >> 1] = pack_half2_ordered(p.x, p.y);
+                        }
                     }
-                    tmem_st16u(tS + 16 * h, packed);
+                    if (h > 0) tmem_st16u(tS + 16 * (h - 1), packed);
                 }
                 const float2 l01 = add2(lp[0], lp[1]), l23 = add2(lp[2], lp[3]);
                 l += (l01.x + l01.y) + (l23.x + l23.y);

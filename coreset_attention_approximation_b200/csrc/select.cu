@@ -73,6 +73,7 @@ struct SelectArgs {
     int32_t bins;      // key bins per caller unit: unit u is bin u % bins of its unit
     int32_t bin_keys;  // keys per bin (pivot indices are reported within the caller's unit)
     const double* kbar;  // centring: mean key of each caller unit ([units / bins][d]), else null
+    uint32_t unit_base;  // Philox unit index of unit 0 (a larger problem's units split across calls)
 };
 
 // Shared-memory plan (bytes) for m rows, r pivots, d dims.
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
                 if (isnan(total)) record_status(status, WC_ERR_NUMERIC);
                 bc.stop = 1;
             } else {
-                const double tau = pivot_uniform(a.seed, (uint32_t)j, (uint32_t)unit) * total;
+                const double tau = pivot_uniform(a.seed, (uint32_t)j, a.unit_base + (uint32_t)unit) * total;
                 double run = 0.0;
                 for (int c = 0; c < a.C; ++c) {
                     const double nxt = run + bsum[c];
@@ -610,6 +611,7 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     a.K = K; a.piv = piv; a.F = F; a.rank = rank;
     a.bins = s.bins;
     a.bin_keys = s.n;
+    a.unit_base = (uint32_t)s.unit_base * (uint32_t)s.bins;   // bin view: unit u * bins + bin
     a.kbar = s.center ? reinterpret_cast<const double*>(ws + L.kbar) : nullptr;
     a.Kt = ws + L.kt;
     a.sync = reinterpret_cast<UnitSync*>(ws + L.sync);

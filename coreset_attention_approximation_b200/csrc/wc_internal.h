@@ -82,6 +82,7 @@ struct Shape {
     int32_t r_pad;         // r rounded up to 128 (whole key tiles of the attention's normaliser column)
     int32_t bins;          // key bins per unit (1: none); select and weights run on the bin view
     int32_t center;        // subtract each unit's mean key before the selection and the weights
+    int32_t unit_base;     // Philox unit index of the caller's first unit (0 for a whole problem)
     // the caller's problem, the same in the unit view and the bin view (sizes the workspace)
     int32_t units_all, n_all, r_all;
 };

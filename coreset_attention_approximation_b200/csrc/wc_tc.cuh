@@ -251,6 +251,14 @@ __device__ __forceinline__ float ex2_ordered(float x) {
     return y;
 }
 
+// fp16 pair {lo, hi} (lo in the low half), kept in program order with the
+// exponentials around it (see ex2_ordered).
+__device__ __forceinline__ uint32_t pack_half2_ordered(float lo, float hi) {
+    uint32_t d;
+    asm volatile("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 // Warpgroup register reallocation (every thread of the warpgroup executes it).
 template <int N>
 __device__ __forceinline__ void reg_claim() {

@@ -5,7 +5,7 @@
 // compressed as V_S = W V.  Here the weights act on [V | 1], so the softmax
 // normaliser is compressed with the values:
 //   C1 = exp(beta K_S K^T) [V | 1]           (gather + exp-GEMM, split over keys)
-//   W  = L^-T (L^-1 C1),  L = F[piv, :rank]  (blocked fp64 triangular solves, 8 columns a block)
+//   W  = L^-T (L^-1 C1),  L = F[piv, :rank]  (blocked fp64 triangular solves, 2-8 columns a block)
 // L L^T = h(K_S, K_S) because the pivot rows of the RPCholesky factor are the
 // Cholesky factor of the kernel matrix on the coreset (in pivot order).
 #include "wc_common.cuh"
@@ -91,6 +91,85 @@ __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t*
 constexpr int kTB = 64;           // rows per diagonal block
 constexpr int kTrsmThreads = 256;
 
+// One 16-entry chunk c of row i's panel segment against the block K = [kb, kb + 64):
+// forward L[i, kb + 16 c + e] (row major; float4 loads when rows start on 16
+// bytes), backward L[kb + 16 c + e, i] (coalesced across the threads' rows).
+template <bool kForward>
+__device__ __forceinline__ void load_chunk(const float* L, int r, int i, int kb, int c, bool vec, float (&v)[16]) {
+    if (kForward) {
+        const float* p = L + (size_t)i * r + kb + 16 * c;
+        if (vec) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(p + e));
+                v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = __ldg(p + e);
+        }
+    } else {
+        const float* p = L + (size_t)(kb + 16 * c) * r + i;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = __ldg(p + (size_t)e * r);
+    }
+}
+
+template <int NC>
+__device__ __forceinline__ void apply_chunk(double (&acc)[NC], const double* Y, int kb, int c, const float (&v)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const double l = (double)v[e];
+        const double* yb = Y + (kb + 16 * c + e) * NC;
+#pragma unroll
+        for (int q = 0; q < NC; ++q) acc[q] = fma(-l, yb[q], acc[q]);
+    }
+}
+
+// Rows i = first, first + stride, ... < end:  Y_i -= L-panel(i) Y_K for a whole
+// 64-row block K.  The update is bound by L2 latency, so each thread keeps the
+// next chunk of L in flight while it applies the current one (the next row's
+// first chunk included).
+template <int NC, bool kForward>
+__device__ void panel_update(double* Y, const float* L, int r, int kb, int first, int end, int stride, bool vec) {
+    if (first >= end) return;
+    float P[16], Q[16];
+    load_chunk<kForward>(L, r, first, kb, 0, vec, P);
+    for (int i = first; i < end; i += stride) {
+        double acc[NC];
+#pragma unroll
+        for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
+        load_chunk<kForward>(L, r, i, kb, 1, vec, Q);
+        apply_chunk<NC>(acc, Y, kb, 0, P);
+        load_chunk<kForward>(L, r, i, kb, 2, vec, P);
+        apply_chunk<NC>(acc, Y, kb, 1, Q);
+        load_chunk<kForward>(L, r, i, kb, 3, vec, Q);
+        apply_chunk<NC>(acc, Y, kb, 2, P);
+        if (i + stride < end) load_chunk<kForward>(L, r, i + stride, kb, 0, vec, P);
+        apply_chunk<NC>(acc, Y, kb, 3, Q);
+#pragma unroll
+        for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
+    }
+}
+
+// The same for a block of bs < 64 rows (the last one), one entry at a time.
+template <int NC, bool kForward>
+__device__ void panel_update_short(double* Y, const float* L, int r, int kb, int bs, int first, int end, int stride) {
+    for (int i = first; i < end; i += stride) {
+        double acc[NC];
+#pragma unroll
+        for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
+        for (int b = 0; b < bs; ++b) {
+            const double l = (double)__ldg(kForward ? L + (size_t)i * r + kb + b : L + (size_t)(kb + b) * r + i);
+            const double* yb = Y + (kb + b) * NC;
+#pragma unroll
+            for (int q = 0; q < NC; ++q) acc[q] = fma(-l, yb[q], acc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
+    }
+}
+
 template <int NC>
 __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restrict__ Lg,
                                                            const int32_t* __restrict__ rank,
@@ -150,34 +229,11 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
             if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
         }
         __syncthreads();
-        // every later row i: Y_i -= L[i, kb .. kb + bs) Y[kb .. kb + bs), 8 entries of L in flight
-        for (int i = kb + bs + tid; i < k; i += kTrsmThreads) {
-            double acc[NC];
-#pragma unroll
-            for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
-            const float* Li = L + (size_t)i * r + kb;
-            for (int b0 = 0; b0 < bs; b0 += 8) {
-                float lv[8];
-                if (rows16 && b0 + 8 <= bs) {
-                    const float4 x = __ldg(reinterpret_cast<const float4*>(Li + b0));
-                    const float4 y = __ldg(reinterpret_cast<const float4*>(Li + b0 + 4));
-                    lv[0] = x.x; lv[1] = x.y; lv[2] = x.z; lv[3] = x.w;
-                    lv[4] = y.x; lv[5] = y.y; lv[6] = y.z; lv[7] = y.w;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) lv[e] = b0 + e < bs ? __ldg(Li + b0 + e) : 0.f;
-                }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const double l = (double)lv[e];
-                    const double* yb = Y + (kb + b0 + e) * NC;
-#pragma unroll
-                    for (int q = 0; q < NC; ++q) acc[q] -= l * yb[q];
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
-        }
+        // every later row i: Y_i -= L[i, kb .. kb + bs) Y[kb .. kb + bs)
+        if (bs == kTB)
+            panel_update<NC, true>(Y, L, r, kb, kb + bs + tid, k, kTrsmThreads, rows16);
+        else
+            panel_update_short<NC, true>(Y, L, r, kb, bs, kb + bs + tid, k, kTrsmThreads);
     }
 
     // ---- backward: L^T x = y
@@ -203,25 +259,10 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
         }
         __syncthreads();
         // every earlier row i: Y_i -= L[kb .. kb + bs, i]^T Y[kb .. kb + bs) (loads coalesced across i)
-        for (int i = tid; i < kb; i += kTrsmThreads) {
-            double acc[NC];
-#pragma unroll
-            for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
-            for (int b0 = 0; b0 < bs; b0 += 8) {
-                float lv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) lv[e] = b0 + e < bs ? __ldg(L + (size_t)(kb + b0 + e) * r + i) : 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const double l = (double)lv[e];
-                    const double* yb = Y + (kb + b0 + e) * NC;
-#pragma unroll
-                    for (int q = 0; q < NC; ++q) acc[q] -= l * yb[q];
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
-        }
+        if (bs == kTB)
+            panel_update<NC, false>(Y, L, r, kb, tid, kb, kTrsmThreads, false);
+        else
+            panel_update_short<NC, false>(Y, L, r, kb, bs, tid, kb, kTrsmThreads);
     }
     __syncthreads();
     for (int e = tid; e < r * nc; e += kTrsmThreads) {
@@ -300,11 +341,16 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
         s.center ? reinterpret_cast<const double*>(ws + L.kk) : nullptr, s.bins, s.n_all, s.beta,
         reinterpret_cast<const double*>(ws + L.shift), status);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
-    // as many right-hand sides per block as shared memory holds for this r
+    // right-hand sides per block: the most that still give 1.5 blocks per SM
+    // (the solve is bound by latency: more blocks keep more loads of L in
+    // flight), within the shared memory that holds them for this r
     const float* Lg = reinterpret_cast<const float*>(ws + L.lg);
     constexpr size_t kMax = 232448;
-    if (trsm_smem<8>(s.r) <= kMax) return launch_trsm_t<8>(s, Lg, rank, Ct, W, status, st);
-    if (trsm_smem<4>(s.r) <= kMax) return launch_trsm_t<4>(s, Lg, rank, Ct, W, status, st);
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    auto enough = [&](int nc) { return (long)s.units * ((s.dv + nc) / nc) * 2 >= 3L * nsm; };
+    if (trsm_smem<8>(s.r) <= kMax && enough(8)) return launch_trsm_t<8>(s, Lg, rank, Ct, W, status, st);
+    if (trsm_smem<4>(s.r) <= kMax && enough(4)) return launch_trsm_t<4>(s, Lg, rank, Ct, W, status, st);
     if (trsm_smem<2>(s.r) <= kMax) return launch_trsm_t<2>(s, Lg, rank, Ct, W, status, st);
     if (trsm_smem<1>(s.r) <= kMax) return launch_trsm_t<1>(s, Lg, rank, Ct, W, status, st);
     return WC_ERR_UNSUPPORTED;

@@ -37,6 +37,7 @@ class WcShape(ctypes.Structure):
         ("dv", ctypes.c_int32), ("r", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("scale", ctypes.c_float), ("eps_stop", ctypes.c_float), ("wait_timeout_ms", ctypes.c_uint32),
         ("seed", ctypes.c_uint64), ("bins", ctypes.c_int32), ("center", ctypes.c_int32),
+        ("unit_base", ctypes.c_int32),
     ]
 
 
@@ -104,10 +105,10 @@ def _stream(stream):
 
 
 def make_shape(batch, hq, hkv, n_k, n_q, d, dv, r, dtype, scale=0.0, eps_stop=0.0, seed=0,
-               wait_timeout_ms=0, bins=1, center=False) -> WcShape:
+               wait_timeout_ms=0, bins=1, center=False, unit_base=0) -> WcShape:
     code = {torch.float32: WC_F32, torch.bfloat16: WC_BF16}.get(dtype, dtype)
     return WcShape(batch, hq, hkv, n_k, n_q, d, dv, r, code, scale, eps_stop, wait_timeout_ms, seed,
-                   int(bins), int(bool(center)))
+                   int(bins), int(bool(center)), int(unit_base))
 
 
 def shape_of(Q, K, V, r, **kw) -> WcShape:

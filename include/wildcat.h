@@ -123,6 +123,12 @@ typedef struct {
                          must be multiples of B */
     int32_t center;   /* 0: keys as given.  1: each unit's mean key is subtracted
                          before the selection and the weights; see "Centring" above */
+    int32_t unit_base; /* >= 0: the Philox unit index of this call's first (batch, kv head)
+                          unit, i.e. the index of its first unit in a larger problem whose
+                          units are split across calls (one call per GPU); 0 for a whole
+                          problem.  Unit u of the call draws its pivots with Philox unit
+                          index unit_base + u (times bins, plus the bin, with bins), so each
+                          unit gets the pivots it gets in one call over the whole problem */
 } wc_shape;
 
 /* Row stride (elements) of F for n_k keys: n_k rounded up to a multiple of 64. */
@@ -143,7 +149,7 @@ size_t wc_forward_workspace_bytes(const wc_shape* shape);
  * overflow), and the pivots, the stop rule and the weights are those of the
  * unshifted kernel; F is the unshifted kernel's factor times exp(-M_u / 2).
  *   d_i = H_ii = exp(beta |k_i|^2 - M_u);   for j = 0 .. r-1:
- *     u_j = Philox4x32-10(ctr = (j, u, 0, 0), key = seed).x0 * 2^-32
+ *     u_j = Philox4x32-10(ctr = (j, unit_base + u, 0, 0), key = seed).x0 * 2^-32
  *     s_j = smallest i with d_0 + ... + d_i > u_j * sum(d)  (inverse CDF)
  *     stop (rank = j) if sum(d) <= 0 or d_{s_j} <= eps_stop * max_i H_ii
  *     F[:, j] = (H[:, s_j] - F[:, :j] F[s_j, :j]^T) / sqrt(d_{s_j}),

@@ -144,7 +144,7 @@ def test_every_entry_point_checks_its_arguments(lib):
     assert lib.wc_forward(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, ok, ok, ok, big, None) == 1
     assert lib.wc_attend_noalloc(ctypes.byref(bad), ok, ok, ok, ok, ok, None) == 1
     # bins and centring: n and r must be multiples of bins; center is 0 or 1
-    for field, value in (("bins", 3), ("bins", -1), ("center", 2)):
+    for field, value in (("bins", 3), ("bins", -1), ("center", 2), ("unit_base", -1)):
         b2 = wildcat.make_shape(1, 2, 1, 512, 16, 64, 64, 32, torch.bfloat16)
         setattr(b2, field, value)
         assert wildcat.workspace_bytes(b2) == 0
