@@ -11,13 +11,20 @@
 namespace wc {
 
 constexpr int kMaxBlocksPerUnit = 512;   // select: thread blocks that share one unit
-constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1 (at most)
-// Keys per partial sum of C1 for units of n keys and r coreset rows:
-// kSplitKeys; or, for heads of at most kSplitKeys keys whose row tiles leave
-// SMs idle, up to 4 splits of whole 128-key tiles (so a few short heads still
+constexpr int kSplitKeys = 4096;         // weights: keys per partial sum of C1 (at least, for long heads)
+// Keys per partial sum of C1 for units of n keys and r coreset rows: for long
+// heads kSplitKeys, doubled while the grid keeps at least 8 waves of blocks
+// (a block's fixed costs, start-up and the store of its partial sums, then
+// weigh less); for heads of at most kSplitKeys keys whose row tiles leave SMs
+// idle, up to 4 splits of whole 128-key tiles (so a few short heads still
 // spread over the GPU, while many short heads keep one block each).
 inline int split_keys(int n, int units, int r) {
-    if (n > kSplitKeys) return kSplitKeys;
+    if (n > kSplitKeys) {
+        const long row_tiles = (long)units * ((r + 127) / 128);
+        int len = kSplitKeys;
+        while (2L * len < n && row_tiles * ((n + 2L * len - 1) / (2L * len)) >= 8L * 148) len *= 2;
+        return len;
+    }
     const long tiles = (long)units * ((r + 127) / 128);
     int want = tiles >= 148 ? 1 : (int)((148 + tiles - 1) / tiles);
     if (want > 4) want = 4;
