@@ -126,29 +126,88 @@ __device__ __forceinline__ void apply_chunk(double (&acc)[NC], const double* Y, 
     }
 }
 
+// acc0 / acc1 (rows i0, i1) -= chunk c of their panel segments times Y_K: each
+// Y_K entry read from shared memory serves both rows.
+template <int NC>
+__device__ __forceinline__ void apply_chunk2(double (&acc0)[NC], double (&acc1)[NC], const double* Y, int kb, int c,
+                                             const float (&v0)[16], const float (&v1)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const double l0 = (double)v0[e], l1 = (double)v1[e];
+        const double* yb = Y + (kb + 16 * c + e) * NC;
+#pragma unroll
+        for (int q = 0; q < NC; ++q) {
+            const double y = yb[q];
+            acc0[q] = fma(-l0, y, acc0[q]);
+            acc1[q] = fma(-l1, y, acc1[q]);
+        }
+    }
+}
+
 // Rows i = first, first + stride, ... < end:  Y_i -= L-panel(i) Y_K for a whole
-// 64-row block K.  The update is bound by L2 latency, so each thread keeps the
-// next chunk of L in flight while it applies the current one (the next row's
-// first chunk included).
-template <int NC, bool kForward>
+// 64-row block K.  The update is bound by load latency and shared-memory
+// reads, not by the fp64 pipe: each thread keeps the next 16-entry chunk of
+// its panel segments in flight while it applies the current one, and with
+// ROWS = 2 takes two rows at a time (i, i + stride), so each Y_K entry it
+// reads from shared memory feeds two fused multiply-adds (twice the registers:
+// one block per SM; worth it when the panels are long, large r).
+template <int NC, bool kForward, int ROWS>
 __device__ void panel_update(double* Y, const float* L, int r, int kb, int first, int end, int stride, bool vec) {
-    if (first >= end) return;
-    float P[16], Q[16];
-    load_chunk<kForward>(L, r, first, kb, 0, vec, P);
-    for (int i = first; i < end; i += stride) {
-        double acc[NC];
+    if (ROWS == 1) {
+        if (first >= end) return;
+        float P[16], Q[16];
+        load_chunk<kForward>(L, r, first, kb, 0, vec, P);
+        for (int i = first; i < end; i += stride) {
+            double acc[NC];
 #pragma unroll
-        for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
-        load_chunk<kForward>(L, r, i, kb, 1, vec, Q);
-        apply_chunk<NC>(acc, Y, kb, 0, P);
-        load_chunk<kForward>(L, r, i, kb, 2, vec, P);
-        apply_chunk<NC>(acc, Y, kb, 1, Q);
-        load_chunk<kForward>(L, r, i, kb, 3, vec, Q);
-        apply_chunk<NC>(acc, Y, kb, 2, P);
-        if (i + stride < end) load_chunk<kForward>(L, r, i + stride, kb, 0, vec, P);
-        apply_chunk<NC>(acc, Y, kb, 3, Q);
+            for (int q = 0; q < NC; ++q) acc[q] = Y[i * NC + q];
+            load_chunk<kForward>(L, r, i, kb, 1, vec, Q);
+            apply_chunk<NC>(acc, Y, kb, 0, P);
+            load_chunk<kForward>(L, r, i, kb, 2, vec, P);
+            apply_chunk<NC>(acc, Y, kb, 1, Q);
+            load_chunk<kForward>(L, r, i, kb, 3, vec, Q);
+            apply_chunk<NC>(acc, Y, kb, 2, P);
+            if (i + stride < end) load_chunk<kForward>(L, r, i + stride, kb, 0, vec, P);
+            apply_chunk<NC>(acc, Y, kb, 3, Q);
 #pragma unroll
-        for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
+            for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
+        }
+        return;
+    }
+    for (int i0 = first; i0 < end; i0 += 2 * stride) {
+        const int i1 = i0 + stride;
+        const bool two = i1 < end;
+        double acc0[NC], acc1[NC];
+#pragma unroll
+        for (int q = 0; q < NC; ++q) {
+            acc0[q] = Y[i0 * NC + q];
+            acc1[q] = two ? Y[i1 * NC + q] : 0.0;
+        }
+        float P0[16], P1[16], Q0[16], Q1[16];
+        load_chunk<kForward>(L, r, i0, kb, 0, vec, P0);
+        if (two) load_chunk<kForward>(L, r, i1, kb, 0, vec, P1);
+        else
+#pragma unroll
+            for (int e = 0; e < 16; ++e) P1[e] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; c += 2) {
+            load_chunk<kForward>(L, r, i0, kb, c + 1, vec, Q0);
+            if (two) load_chunk<kForward>(L, r, i1, kb, c + 1, vec, Q1);
+            else
+#pragma unroll
+                for (int e = 0; e < 16; ++e) Q1[e] = 0.f;
+            apply_chunk2<NC>(acc0, acc1, Y, kb, c, P0, P1);
+            if (c + 2 < 4) {
+                load_chunk<kForward>(L, r, i0, kb, c + 2, vec, P0);
+                if (two) load_chunk<kForward>(L, r, i1, kb, c + 2, vec, P1);
+            }
+            apply_chunk2<NC>(acc0, acc1, Y, kb, c + 1, Q0, Q1);
+        }
+#pragma unroll
+        for (int q = 0; q < NC; ++q) {
+            Y[i0 * NC + q] = acc0[q];
+            if (two) Y[i1 * NC + q] = acc1[q];
+        }
     }
 }
 
@@ -170,7 +229,7 @@ __device__ void panel_update_short(double* Y, const float* L, int r, int kb, int
     }
 }
 
-template <int NC>
+template <int NC, int ROWS>
 __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restrict__ Lg,
                                                            const int32_t* __restrict__ rank,
                                                            const double* __restrict__ Ct, float* W, int r, int dv,
@@ -231,7 +290,7 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
         __syncthreads();
         // every later row i: Y_i -= L[i, kb .. kb + bs) Y[kb .. kb + bs)
         if (bs == kTB)
-            panel_update<NC, true>(Y, L, r, kb, kb + bs + tid, k, kTrsmThreads, rows16);
+            panel_update<NC, true, ROWS>(Y, L, r, kb, kb + bs + tid, k, kTrsmThreads, rows16);
         else
             panel_update_short<NC, true>(Y, L, r, kb, bs, kb + bs + tid, k, kTrsmThreads);
     }
@@ -260,7 +319,7 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
         __syncthreads();
         // every earlier row i: Y_i -= L[kb .. kb + bs, i]^T Y[kb .. kb + bs) (loads coalesced across i)
         if (bs == kTB)
-            panel_update<NC, false>(Y, L, r, kb, tid, kb, kTrsmThreads, false);
+            panel_update<NC, false, ROWS>(Y, L, r, kb, tid, kb, kTrsmThreads, false);
         else
             panel_update_short<NC, false>(Y, L, r, kb, bs, tid, kb, kTrsmThreads);
     }
@@ -280,10 +339,11 @@ template <int NC>
 wc_status launch_trsm_t(const Shape& s, const float* Lg, const int32_t* rank, const double* Ct, float* W,
                         int* status, cudaStream_t st) {
     const size_t smem = trsm_smem<NC>(s.r);
-    if (cudaFuncSetAttribute(trsm_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    // two rows per thread where the panels are long (they hold 512 rows on average from r = 1024)
+    auto kern = s.r >= 1024 ? trsm_kernel<NC, 2> : trsm_kernel<NC, 1>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return WC_ERR_CUDA;
-    trsm_kernel<NC><<<dim3((s.dv + 1 + NC - 1) / NC, s.units), kTrsmThreads, smem, st>>>(Lg, rank, Ct, W, s.r, s.dv,
-                                                                                        status);
+    kern<<<dim3((s.dv + 1 + NC - 1) / NC, s.units), kTrsmThreads, smem, st>>>(Lg, rank, Ct, W, s.r, s.dv, status);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -341,18 +401,29 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
         s.center ? reinterpret_cast<const double*>(ws + L.kk) : nullptr, s.bins, s.n_all, s.beta,
         reinterpret_cast<const double*>(ws + L.shift), status);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
-    // right-hand sides per block: the most that still give 1.5 blocks per SM
-    // (the solve is bound by latency: more blocks keep more loads of L in
-    // flight), within the shared memory that holds them for this r
+    // right-hand sides per block: 8 (the fewest re-reads of L, and each block
+    // repeats the serial diagonal solves), fewer only while the blocks would
+    // fill less than half of the GPU (one block per SM with two rows per
+    // thread, two with one), within the shared memory that holds the columns
+    // for this r
     const float* Lg = reinterpret_cast<const float*>(ws + L.lg);
     constexpr size_t kMax = 232448;
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    auto enough = [&](int nc) { return (long)s.units * ((s.dv + nc) / nc) * 2 >= 3L * nsm; };
-    if (trsm_smem<8>(s.r) <= kMax && enough(8)) return launch_trsm_t<8>(s, Lg, rank, Ct, W, status, st);
-    if (trsm_smem<4>(s.r) <= kMax && enough(4)) return launch_trsm_t<4>(s, Lg, rank, Ct, W, status, st);
-    if (trsm_smem<2>(s.r) <= kMax) return launch_trsm_t<2>(s, Lg, rank, Ct, W, status, st);
-    if (trsm_smem<1>(s.r) <= kMax) return launch_trsm_t<1>(s, Lg, rank, Ct, W, status, st);
+    auto smem_ok = [&](int nc) {
+        return (nc == 8 ? trsm_smem<8>(s.r) : nc == 4 ? trsm_smem<4>(s.r) : nc == 2 ? trsm_smem<2>(s.r)
+                                                                                  : trsm_smem<1>(s.r)) <= kMax;
+    };
+    int best = 0;
+    for (int nc : {8, 4, 2, 1}) {
+        if (!smem_ok(nc)) continue;
+        best = nc;
+        if ((long)s.units * ((s.dv + nc) / nc) * 2 >= (long)nsm * (s.r >= 1024 ? 1 : 2)) break;
+    }
+    if (best == 8) return launch_trsm_t<8>(s, Lg, rank, Ct, W, status, st);
+    if (best == 4) return launch_trsm_t<4>(s, Lg, rank, Ct, W, status, st);
+    if (best == 2) return launch_trsm_t<2>(s, Lg, rank, Ct, W, status, st);
+    if (best == 1) return launch_trsm_t<1>(s, Lg, rank, Ct, W, status, st);
     return WC_ERR_UNSUPPORTED;
 }
 
