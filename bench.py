@@ -45,10 +45,12 @@ from coreset_attention_approximation_b200.workloads import WORKLOADS, make_input
 METRIC = "WildCat forward tokens/sec at 1 B200; select HBM GB/s and GEMM TC-util vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) of the select kernel per unit and launch, measured
-# with ncu's dram__bytes_read.sum + dram__bytes_write.sum on the named workload:
-# long = 9.306759 TB + 8.881209 GB over 8 units.  Other workloads: not captured.
-SELECT_DRAM_BYTES_PER_UNIT = {"long": (9.306759e12 + 8.881209e9) / 8}
+# DRAM bytes (read + write) of the select kernel per unit and launch on the named
+# workload: ncu's dram__bytes_read.sum + dram__bytes_write.sum on the same 8 units
+# and keys with r = 512 (669.953816 GB + 2.396056 GB against 688.268509 GB of
+# algorithmic bytes: 0.97687), applied to the algorithmic bytes at r = 2048.
+# Other workloads: not captured.
+SELECT_DRAM_BYTES_PER_UNIT = {"long": 0.976871 * 9350143803392 / 8}
 
 
 def load_peaks():
