@@ -50,8 +50,7 @@ constexpr int kGroup = 2;
 // Rows per block are a multiple of 128, so every block's slice of F (fp32) and
 // of the transposed keys (bf16) starts on a 256-byte boundary: blocks whose
 // slices did not streamed their share about 6 % slower, and every step waits
-// for the slowest block of the unit.  A multiple of 64 (F slices still on 256
-// bytes) is taken where it balances the SMs' rows better (few units).
+// for the slowest block of the unit.
 constexpr int kRowAlign = 128;
 
 struct SelectArgs {
@@ -66,7 +65,7 @@ struct SelectArgs {
     int64_t ldf;
     int32_t n, d, r;
     int32_t C;      // blocks per unit
-    int32_t m;      // rows per block (multiple of kRowAlign / 2)
+    int32_t m;      // rows per block (multiple of kRowAlign)
     int32_t unit0;  // first unit of this wave
     double beta, eps;
     uint64_t seed;
@@ -505,13 +504,9 @@ struct SelectPlan {
     int per_sm = 0;     // of those, a SM's
 };
 
-// Blocks per unit.  The blocks of a unit wait on each other, so every block of
-// the launch must be co-resident, and a step lasts as long as the SM with the
-// most rows: among the block counts that put p = 1, 2, ... blocks on each SM
-// (rows per block a multiple of 128, or of 64 where that balances the SMs
-// better), take the one whose busiest SM holds the fewest rows, ties to more
-// blocks per SM (more loads in flight).  With no co-resident choice, the fewest
-// blocks the shared memory allows, in co-resident waves.
+// Most blocks per unit such that every block of the launch is co-resident
+// (they wait on each other), at >= 256 rows per block; else the fewest blocks
+// the shared memory allows, in co-resident waves.
 template <typename T, typename TK, int NT>
 wc_status plan_select(const Shape& s, int nsm, int max_smem, int m_max, SelectPlan* p) {
     auto kern = rpcholesky_kernel<T, TK, NT>;
@@ -523,42 +518,27 @@ wc_status plan_select(const Shape& s, int nsm, int max_smem, int m_max, SelectPl
             return 0;
         return b;
     };
-    auto rows_for = [&](long C, int align) { return (int)(((s.n + C - 1) / C + align - 1) / align * align); };
+    auto rows_for = [&](int C) { return ((s.n + C - 1) / C + kRowAlign - 1) / kRowAlign * kRowAlign; };
     const int c_min = (s.n + m_max - 1) / m_max;
     int c_hi = (s.n + 255) / 256;
     if (c_hi > kMaxBlocksPerUnit) c_hi = kMaxBlocksPerUnit;
     if (c_hi < c_min) c_hi = c_min;
-    long best_cost = -1;
-    int best_m = 0, best_bps = 0;
-    long best_blocks = 0;
-    for (int per = 1; per <= 16; ++per) {
-        const long target = (long)per * nsm / s.units;
-        for (long c = target; c <= target + 1; ++c) {
-            if (c < 2 || c < c_min || c > c_hi) continue;
-            for (int align : {kRowAlign, kRowAlign / 2}) {
-                const int m = rows_for(c, align);
-                if (m > m_max) continue;
-                const long blocks = (long)s.units * ((s.n + m - 1) / m);
-                const int bps = blocks_per_sm(m);
-                if (bps < 1 || blocks > (long)nsm * bps) continue;
-                const long cost = (blocks + nsm - 1) / nsm * m;   // rows of the busiest SM
-                if (best_cost < 0 || cost < best_cost || (cost == best_cost && blocks > best_blocks)) {
-                    best_cost = cost;
-                    best_m = m;
-                    best_bps = bps;
-                    best_blocks = blocks;
-                }
-            }
+    int m = rows_for(c_min);
+    int bps = blocks_per_sm(m);
+    for (int c = c_hi; c > c_min; --c) {
+        const int mc = rows_for(c);
+        const int ce = (s.n + mc - 1) / mc;
+        const int bc = blocks_per_sm(mc);
+        if ((long)s.units * ce <= (long)nsm * bc) {
+            m = mc;
+            bps = bc;
+            break;
         }
     }
-    if (best_cost < 0) {
-        best_m = rows_for(c_min, kRowAlign);
-        best_bps = blocks_per_sm(best_m);
-    }
-    p->m = best_m;
-    p->C = (s.n + best_m - 1) / best_m;
-    p->per_sm = best_bps;
-    p->cap = (long)nsm * best_bps;
+    p->m = m;
+    p->C = (s.n + m - 1) / m;
+    p->per_sm = bps;
+    p->cap = (long)nsm * bps;
     return WC_OK;
 }
 
