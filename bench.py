@@ -509,7 +509,7 @@ def kernel_breakdown(step):
         if "wc::" in name:
             out["launches"] += 1          # this library's kernels (namespace wc)
         short = None
-        m = re.search(r"expmm_(tc|simt)_kernel<[^>]*?(\d)>", name)
+        m = re.search(r"expmm_(tc|simt|pair)_kernel<[^>]*?(\d)>", name)
         if m:
             # modes 0, 2: the weights' partial sums; 1: attention; 3: attention over a key split
             short = "attend_gemm" if m.group(2) in ("1", "3") else "weights_gemm"

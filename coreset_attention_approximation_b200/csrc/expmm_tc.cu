@@ -83,6 +83,18 @@ constexpr uint64_t kTcTimeoutNs = 4000000000ull;
 #ifndef WC_HANDOFF_QUARTER
 #define WC_HANDOFF_QUARTER 0
 #endif
+// Attention over short coresets (at most two 128-key tiles) with at least two
+// query tiles a head runs on the paired-row-tile kernel (expmm_pair_kernel):
+// there a CTA's fixed start-up and store dominate, and pairing halves them per
+// row tile (measured 1.37-1.44x on the ViT- and diffusion-shaped heads).  With
+// more key tiles it was slower than expmm_tc_kernel (0.51-0.53 against 0.57-0.60
+// of the bf16 burst figure on the long workload's heads: the issuing thread
+// waits for PV_p(t) before S_p(t + 1) may overwrite P_p(t)), and so are the
+// weights.  WC_PAIR_TILES = 0 turns it off.
+#ifndef WC_PAIR_TILES
+#define WC_PAIR_TILES 1
+#endif
+constexpr bool kPairTiles = WC_PAIR_TILES != 0;
 constexpr int kFmaExpCols = WC_EXP2_FMA_COLS;
 constexpr int kHandQuarter = WC_HANDOFF_QUARTER;
 constexpr int kFmaExpSpread = WC_EXP2_FMA_SPREAD;
@@ -612,6 +624,429 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 2) tmem_dealloc<512>(tmem);
 }
 
+// ---------------------------------------------------------------------------
+// Paired row tiles: one CTA computes two 128-row tiles of A (256 rows) against
+// the same key and value tiles, each loaded once for both.  Softmax warps 4..7
+// own row tile 0 and warps 8..11 row tile 1: a warp holds whole rows, so it
+// keeps its own running maximum (no hand-over between warps), and the two
+// warps of an SM sub-partition run their exponentials side by side on the
+// exponential unit.  One thread issues every MMA, interleaving the two tiles
+// so that each softmax has the other tile's MMAs to hide behind:
+//   S0(0) S1(0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ...
+// S_p(t+1) overwrites the TMEM columns from which PV_p(t) reads P_p(t); the
+// issuing thread waits for PV_p(t) to complete first.
+// TMEM: S_p at columns 128 p (P_p as fp16 pairs over its first 64 columns),
+// O_p at 256 + DV p.  Modes: kExpmmPartial (the weights' partial sums) and
+// kExpmmRownorm (attention).  The epilogue stages both tiles' rows in the
+// operand rings (idle once the last MMA has completed) and stores them with
+// bulk asynchronous copies.
+template <int D, int DV>
+struct SmemPair {
+    static constexpr uint32_t kA = BM * D * 2;
+    static constexpr uint32_t kB = BN * D * 2;
+    static constexpr uint32_t kC = BN * DV * 2;
+    // stages of the key and value rings: as many as fit beside both row tiles
+    static constexpr int kStages = 2 * kA + 4 * (kB + kC + BN * 4) + 4096 <= 232448   ? 4
+                                   : 2 * kA + 3 * (kB + kC + BN * 4) + 4096 <= 232448 ? 3
+                                                                                       : 2;
+    static constexpr uint32_t A = 0;                              // [2] row tiles
+    static constexpr uint32_t B0 = 2 * kA;                        // [kStages] key tiles
+    static constexpr uint32_t C0 = B0 + kStages * kB;             // [kStages] value tiles
+    static constexpr uint32_t Wv = C0 + kStages * kC;             // [kStages][BN] normaliser weights
+    static constexpr uint32_t Bar = Wv + kStages * BN * 4;
+    static constexpr uint32_t kAlloc = Bar + 256;
+    // epilogue staging of row tile p (rows c1_row(DV) floats apart) over the idle rings
+    static constexpr uint32_t kStageBytes = (BM * c1_row(DV) * 4 + 1023) / 1024 * 1024;
+    static_assert(2 * kStageBytes <= Wv, "both row tiles stage in the operand rings");
+    static_assert(kAlloc <= 232448, "shared memory per block");
+};
+
+template <int D, int DV, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    expmm_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                      const __grid_constant__ CUtensorMap mapC, const TcArgs args) {
+    using L = SmemPair<D, DV>;
+    constexpr int NR = L::kStages;
+    constexpr bool kQueries = MODE == kExpmmRownorm;
+    static_assert(MODE == kExpmmPartial || MODE == kExpmmRownorm, "paired tiles: weights or attention");
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw;
+    if (smem_u32(sm) & 1023u) {
+        if (threadIdx.x == 0) record_status(args.status, WC_ERR_UNSUPPORTED);
+        return;
+    }
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::Bar);
+    uint64_t* fullB = bars;                   // [NR]
+    uint64_t* emptyB = fullB + NR;            // [NR]
+    uint64_t* fullC = emptyB + NR;            // [NR]
+    uint64_t* emptyC = fullC + NR;            // [NR]
+    uint64_t* a_full = emptyC + NR;
+    uint64_t* s_full = a_full + 1;            // [2] per row tile
+    uint64_t* p_full = s_full + 2;            // [2]
+    uint64_t* pv_done = p_full + 2;           // [2]
+    uint64_t* drain = pv_done + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int z = blockIdx.z;
+    int unit, a_valid, b_lo, b_hi, split = 0, a_row0;
+    if (!kQueries) {
+        unit = z;
+        a_valid = args.rank[unit];
+        if (!in_bounds(a_valid >= 0 && a_valid <= args.r, args.status)) return;
+        split = blockIdx.y;
+        b_lo = split * args.split_len;
+        b_hi = min(args.b_rows, b_lo + args.split_len);
+        a_row0 = unit * args.a_head_rows + blockIdx.x * 2 * BM;
+    } else {
+        const int hkv = args.hq / args.group;
+        unit = (z / args.hq) * hkv + (z % args.hq) / args.group;
+        a_valid = args.a_rows;
+        const int b_all = args.all_keys ? args.b_rows : args.rank[unit];
+        if (!in_bounds(b_all >= 0 && b_all <= args.b_rows, args.status)) return;
+        b_lo = 0;
+        b_hi = b_all;
+        a_row0 = z * args.a_head_rows + blockIdx.x * 2 * BM;
+    }
+    const int a0 = blockIdx.x * 2 * BM;
+    if (a0 >= a_valid) return;
+    const int T = b_hi > b_lo ? (b_hi - b_lo + BN - 1) / BN : 0;
+    const int b_row0 = unit * args.b_rows + b_lo;
+
+    if (tid == 0) {
+        for (int i = 0; i < NR; ++i) {
+            mbar_init(&fullB[i], 1);
+            mbar_init(&emptyB[i], 1);
+            mbar_init(&fullC[i], 1);
+            mbar_init(&emptyC[i], 1);
+        }
+        mbar_init(a_full, 1);
+        for (int p = 0; p < 2; ++p) {
+            mbar_init(&s_full[p], 1);
+            mbar_init(&p_full[p], 4);
+            mbar_init(&pv_done[p], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 2) tmem_alloc<512>(tmem_slot);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 4) {
+        reg_release<kRegsSide>();
+        if (warp <= 1) {
+            // ------------------------------------------------------------ TMA producers
+            // warp 0: both row tiles of A, then the key tiles; warp 1: the value tiles (and w)
+            const bool keys = warp == 0;
+            if (lane == 0 && T > 0) {
+                if (keys) {
+                    tma_prefetch(&mapA);
+                    tma_prefetch(&mapB);
+                    mbar_expect_tx(a_full, 2 * L::kA);
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int c = 0; c < D / 64; ++c)
+                            tma_load_2d(sm + L::A + p * L::kA + c * (BM * 128), &mapA, a_full, c * 64, a_row0 + p * BM);
+                } else {
+                    tma_prefetch(&mapC);
+                }
+                uint64_t* fl = keys ? fullB : fullC;
+                uint64_t* em = keys ? emptyB : emptyC;
+                int issued = 0;
+                for (int t = 0; t < T; ++t) {
+                    const int s = t % NR;
+                    if (t >= NR && !mbar_wait(&em[s], ((t / NR) - 1) & 1, abort_flag, args.status, kTcTimeoutNs))
+                        break;
+                    const int brow = b_row0 + t * BN;
+                    if (keys) {
+                        mbar_expect_tx(&fl[s], L::kB);
+                        unsigned char* st = sm + L::B0 + s * L::kB;
+#pragma unroll
+                        for (int c = 0; c < D / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapB, &fl[s], c * 64, brow);
+                    } else {
+                        mbar_expect_tx(&fl[s], L::kC + (kQueries ? BN * 4 : 0));
+                        unsigned char* st = sm + L::C0 + s * L::kC;
+#pragma unroll
+                        for (int c = 0; c < DV / 64; ++c) tma_load_2d(st + c * (BN * 128), &mapC, &fl[s], c * 64, brow);
+                        if (kQueries)
+                            bulk_load(sm + L::Wv + s * BN * 4, args.wn + (size_t)unit * args.r_pad + b_lo + t * BN,
+                                      BN * 4, &fl[s]);
+                    }
+                    issued = t + 1;
+                }
+                if (*abort_flag) {
+                    const uint64_t t0 = global_ns();
+                    while (keys && !mbar_try_wait(a_full, 0) && global_ns() - t0 < 100000000ull) {
+                    }
+                    for (int t = issued - NR > 0 ? issued - NR : 0; t < issued; ++t) {
+                        const uint64_t t1 = global_ns();
+                        while (!mbar_try_wait(&fl[t % NR], (t / NR) & 1) && global_ns() - t1 < 100000000ull) {
+                        }
+                    }
+                }
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------------------------ MMA issuer (both row tiles)
+            if (lane == 0) {
+                constexpr uint32_t idS = idesc_f16(BM, BN, 1, 1, 0, 0);   // bf16 x bf16, both K-major
+                constexpr uint32_t idO = idesc_f16(BM, DV, 0, 0, 0, 1);   // f16 P (TMEM) x f16 C (MN-major)
+                const uint64_t dA = sdesc_sw128(smem_u32(sm + L::A), 16, 1024);
+                const uint64_t dB = sdesc_sw128(smem_u32(sm + L::B0), 16, 1024);
+                const uint64_t dC = sdesc_sw128(smem_u32(sm + L::C0), BN * 128, 1024);
+                auto issue_s = [&](int p, int t) {
+                    const uint64_t a = dA + (uint64_t)((p * L::kA) >> 4);
+                    const uint64_t b = dB + (uint64_t)(((t % NR) * L::kB) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t oa = (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
+                        const uint64_t ob = (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
+                        mma_f16_ss(tmem + p * BN, a + oa, b + ob, idS, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[p]);
+                };
+                auto issue_pv = [&](int p, int t) {
+                    const uint64_t c = dC + (uint64_t)(((t % NR) * L::kC) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_f16_ts(tmem + 2 * BN + p * DV, tmem + p * BN + 8 * kk, c + (uint64_t)((kk * 16 * 128) >> 4),
+                                   idO, (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&pv_done[p]);
+                };
+                bool ok = T > 0 && mbar_wait(a_full, 0, abort_flag, args.status, kTcTimeoutNs);
+                if (ok) ok = mbar_wait(&fullB[0], 0, abort_flag, args.status, kTcTimeoutNs);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0, 0);
+                    issue_s(1, 0);
+                    mma_commit(&emptyB[0]);
+                }
+                for (int t = 0; ok && t < T; ++t) {
+                    const bool more = t + 1 < T;
+                    ok = mbar_wait(&fullC[t % NR], (t / NR) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (ok) ok = mbar_wait(&p_full[0], t & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(0, t);
+                    if (more) {
+                        ok = mbar_wait(&fullB[(t + 1) % NR], ((t + 1) / NR) & 1, abort_flag, args.status, kTcTimeoutNs);
+                        // S_0(t + 1) overwrites the columns PV_0(t) reads P_0(t) from
+                        if (ok) ok = mbar_wait(&pv_done[0], t & 1, abort_flag, args.status, kTcTimeoutNs);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(0, t + 1);
+                    }
+                    ok = mbar_wait(&p_full[1], t & 1, abort_flag, args.status, kTcTimeoutNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, t);
+                    mma_commit(&emptyC[t % NR]);
+                    if (more) {
+                        ok = mbar_wait(&pv_done[1], t & 1, abort_flag, args.status, kTcTimeoutNs);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(1, t + 1);
+                        mma_commit(&emptyB[(t + 1) % NR]);
+                    }
+                }
+                mma_commit(drain);
+            }
+        }
+    } else {
+        reg_claim<kRegsSoftmax>();
+        // ------------------------------------------------------------ softmax + epilogue of row tile p
+        const int p = (warp - 4) >> 2;          // row tile of this warp
+        const int q = warp & 3;                 // TMEM lanes 32 q .. 32 q + 31
+        const int row = q * 32 + lane;
+        const uint32_t lanes = (uint32_t)(q * 32) << 16;
+        const uint32_t tS = tmem + p * BN + lanes;
+        const uint32_t tO = tmem + 2 * BN + p * DV + lanes;
+        const float cb = args.cb;
+        const float2 cb2 = make_float2(cb, cb);
+        float mO = -INFINITY;                   // this row's reference (log2 units)
+        float l = 0.f;                          // its normaliser share, relative to mO
+        bool ok = true;
+        for (int t = 0; t < T; ++t) {
+            ok = ok && mbar_wait(&s_full[p], t & 1, abort_flag, args.status, kTcTimeoutNs);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            const int valid = b_hi - (b_lo + t * BN);
+            float sv[BN];
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 4; ++h) tmem_ld32(tS + 32 * h, sv + 32 * h);
+            tmem_wait_ld();
+            if (valid < BN) {
+#pragma unroll
+                for (int j = 0; j < BN; ++j)
+                    if (j >= valid) sv[j] = -INFINITY;
+            }
+            float mq[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mq[i] = sv[i];
+#pragma unroll
+            for (int j = 8; j < BN; j += 2) mq[(j >> 1) & 7] = fmax3(mq[(j >> 1) & 7], sv[j], sv[j + 1]);
+            const float mt = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7])) * cb;
+            const bool grow = __any_sync(0xffffffffu, mt > mO + kRescale);
+            if (grow) {
+                const float mn = fmaxf(mO, mt);
+                const float sc = (mO == -INFINITY) ? 0.f : ex2(mO - mn);
+                l *= sc;
+                if (t > 0) {
+                    // O holds key tiles 0..t-1 in the old reference: rescale once PV(t - 1) has landed
+                    ok = mbar_wait(&pv_done[p], (t - 1) & 1, abort_flag, args.status, kTcTimeoutNs);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int c0 = 0; c0 < DV; c0 += 32) {
+                        float o[32];
+                        tmem_ld32(tO + c0, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= sc;
+                        tmem_st32(tO + c0, o);
+                    }
+                    tmem_wait_st();
+                }
+                mO = mn;
+            }
+            if (kQueries) {
+                // w arrives with the value tile; this stage cannot be reloaded before PV_1(t)
+                ok = mbar_wait(&fullC[t % NR], (t / NR) & 1, abort_flag, args.status, kTcTimeoutNs);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            const float* wv = reinterpret_cast<const float*>(sm + L::Wv + (t % NR) * BN * 4);
+            const float2 nm2 = make_float2(-mO, -mO);
+            float2 lp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
+            // quarter h's exponentials between the packing of quarter h - 1 (see expmm_tc_kernel)
+#pragma unroll
+            for (int h = 0; h <= 4; ++h) {
+                uint32_t packed[16];
+                float w[kQueries ? 32 : 1];
+                if (kQueries && h > 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 f = lds_f4_ordered(wv + 32 * (h - 1) + j);
+                        w[j] = f.x;
+                        w[j + 1] = f.y;
+                        w[j + 2] = f.z;
+                        w[j + 3] = f.w;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    if (h < 4) {
+                        const int c = 32 * h + j;
+                        const float2 x2 = fma2(make_float2(sv[c], sv[c + 1]), cb2, nm2);
+                        float2 pp;
+                        if (fma_exp_col(c)) {
+                            pp = exp2_fma2(x2);
+                        } else {
+                            pp.x = ex2_ordered(x2.x);
+                            pp.y = ex2_ordered(x2.y);
+                        }
+                        sv[c] = pp.x;
+                        sv[c + 1] = pp.y;
+                    }
+                    if (h > 0) {
+                        const int c = 32 * (h - 1) + j;
+                        const float2 pp = make_float2(sv[c], sv[c + 1]);
+                        if (kQueries)
+                            lp[(j >> 1) & 3] = fma2(pp, make_float2(w[j], w[j + 1]), lp[(j >> 1) & 3]);
+                        else
+                            lp[(j >> 1) & 3] = add2(lp[(j >> 1) & 3], pp);
+                        packed[j >> 1] = pack_half2_ordered(pp.x, pp.y);
+                    }
+                }
+                if (h > 0) tmem_st16u(tS + 16 * (h - 1), packed);
+            }
+            const float2 l01 = add2(lp[0], lp[1]), l23 = add2(lp[2], lp[3]);
+            l += (l01.x + l01.y) + (l23.x + l23.y);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[p]);
+        }
+
+        // ------------------------------------------------------------ epilogue of row tile p
+        // once every MMA has completed the operand rings are idle: row tile p stages its
+        // rows (c1_row(DV) floats apart) at L::kStageBytes p, then bulk copies store them
+        const float4* s4 = reinterpret_cast<const float4*>(args.sigma + (size_t)unit * DV);
+        {
+            const uint64_t t0 = global_ns();
+            bool drained = false;
+            while (!(drained = mbar_try_wait(drain, 0)) && global_ns() - t0 < 2000000000ull) {
+            }
+            if (!drained) {
+                record_status(args.status, WC_ERR_TIMEOUT);
+                ok = false;
+            }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) tc_fence_after();
+        constexpr int SST = c1_row(DV);
+        float* stg = reinterpret_cast<float*>(sm + p * L::kStageBytes);
+        const bool have_o = ok && T > 0;
+        const float inv = kQueries ? 1.f / l : 1.f;
+        float* srow = stg + row * SST;
+#pragma unroll
+        for (int c0 = 0; c0 < DV; c0 += 32) {
+            float o[32];
+            if (have_o) {
+                tmem_ld32(tO + c0, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = 0.f;
+            }
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+                float4 v = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                if (kQueries) {
+                    const float4 g = __ldg(s4 + (c0 + c) / 4);   // the column scales of the fp16 weights
+                    v.x *= g.x * inv;
+                    v.y *= g.y * inv;
+                    v.z *= g.z * inv;
+                    v.w *= g.w * inv;
+                }
+                *reinterpret_cast<float4*>(srow + c0 + c) = v;
+            }
+        }
+        if (!kQueries) *reinterpret_cast<float2*>(srow + DV) = make_float2(l, mO * kLn2);
+        fence_async_smem();
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + p) : "memory");   // the row tile's 4 warps have staged
+        const int ap = a0 + p * BM;
+        const int rows = min(BM, a_valid - ap);
+        const int st = tid - 4 * 32 - p * 128;  // 0 .. 127 within the row tile
+        if (ok && rows > 0) {
+            if (!kQueries && st == 0) {
+                const size_t prow = ((size_t)unit * args.nsplit + split) * args.r + ap;
+                bulk_store(static_cast<float*>(args.out) + prow * SST, stg, (uint32_t)(rows * SST * 4));
+                bulk_commit();
+                bulk_wait_read_all();
+            }
+            if (kQueries && st < rows) {
+                bulk_store(static_cast<float*>(args.out) + ((size_t)z * args.a_rows + ap + st) * DV, stg + st * SST,
+                           (uint32_t)(DV * 4));
+                bulk_commit();
+                bulk_wait_read_all();
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc<512>(tmem);
+}
+
 // Key-split attention: row q of query head h from its splits' partial rows
 // (O_s | l_s | m_s, m in natural-log units):
 //   out[h][q][c] = sum_s e_s O_s[c] / sum_s e_s l_s,  e_s = exp(m_s - max_s m_s).
@@ -773,6 +1208,31 @@ wc_status launch_tc_t(const CUtensorMap& A, const CUtensorMap& B, const CUtensor
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
+template <int D, int DV, int MODE>
+wc_status launch_pair_t(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& C, const TcArgs& a,
+                        dim3 grid, cudaStream_t st) {
+    using L = SmemPair<D, DV>;
+    auto kern = expmm_pair_kernel<D, DV, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc) != cudaSuccess)
+        return WC_ERR_CUDA;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return WC_ERR_CUDA;
+    if (fa.numRegs < kRegsLaunch) return WC_ERR_UNSUPPORTED;
+    kern<<<grid, kThreads, L::kAlloc, st>>>(A, B, C, a);
+    return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+// Paired row tiles (two 128-row tiles of A per CTA): grid.x counts pairs.
+template <int MODE>
+wc_status launch_pair(int d, int dv, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& C,
+                      const TcArgs& a, dim3 grid, cudaStream_t st) {
+    if (d == 64 && dv == 64) return launch_pair_t<64, 64, MODE>(A, B, C, a, grid, st);
+    if (d == 64 && dv == 128) return launch_pair_t<64, 128, MODE>(A, B, C, a, grid, st);
+    if (d == 128 && dv == 64) return launch_pair_t<128, 64, MODE>(A, B, C, a, grid, st);
+    if (d == 128 && dv == 128) return launch_pair_t<128, 128, MODE>(A, B, C, a, grid, st);
+    return WC_ERR_UNSUPPORTED;
+}
+
 template <int MODE>
 wc_status launch_tc(int d, int dv, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& C,
                     const TcArgs& a, dim3 grid, cudaStream_t st) {
@@ -791,6 +1251,9 @@ wc_status launch_exp2_selftest(const float* x, float* y, int64_t n, int method, 
     exp2_selftest_kernel<<<blocks, 256, 0, st>>>(x, y, n, method);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
+
+// the paired kernel's attention rule (see kPairTiles)
+bool use_pair_tiles(const Shape& s) { return kPairTiles && s.r <= 2 * BN && s.nq > BM; }
 
 int attend_splits(const Shape& s) {
     // the attention's query tiles alone fill the GPU: no split
@@ -883,6 +1346,10 @@ wc_status launch_attend_tc(const Shape& s, const void* Q, const void* Ks, const 
     a.cb = (float)(s.beta * 1.4426950408889634);
     const int ns = attend_splits(s);
     if (ns <= 1) {
+        if (use_pair_tiles(s)) {
+            dim3 pgrid((s.nq + 2 * BM - 1) / (2 * BM), 1, s.batch * s.hq);
+            return launch_pair<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, pgrid, st);
+        }
         dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
         return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
     }
@@ -932,6 +1399,10 @@ wc_status launch_attend_tc_at(const Shape& s, const void* Q, const void* Ks, con
     a.group = s.hq / s.hkv;
     a.all_keys = s.bins > 1;
     a.cb = (float)(s.beta * 1.4426950408889634);
+    if (use_pair_tiles(s)) {
+        dim3 pgrid((s.nq + 2 * BM - 1) / (2 * BM), 1, s.batch * s.hq);
+        return launch_pair<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, pgrid, st);
+    }
     dim3 grid((s.nq + TILES * BM - 1) / (TILES * BM), 1, s.batch * s.hq);
     return launch_tc<kExpmmRownorm>(s.d, s.dv, mA, mB, mC, a, grid, st);
 }
