@@ -515,7 +515,7 @@ def kernel_breakdown(step):
             short = "attend_gemm" if m.group(2) in ("1", "3") else "weights_gemm"
         else:
             for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
-                             ("merge_c1", "merge_c1"), ("trsm_kernel", "solve"),
+                             ("merge_c1", "merge_c1"), ("trsm_", "solve"),
                              ("weights_prep", "w_prep"), ("key_shift", "shift"),
                              ("attend_combine", "attend_combine")):
                 if key in name:

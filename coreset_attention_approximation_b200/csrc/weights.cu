@@ -153,7 +153,7 @@ __device__ __forceinline__ void apply_chunk2(double (&acc0)[NC], double (&acc1)[
 // one block per SM; worth it when the panels are long, large r).
 template <int NC, bool kForward, int ROWS>
 __device__ void panel_update(double* Y, const float* L, int r, int kb, int first, int end, int stride, bool vec) {
-    if (ROWS == 1) {
+    if constexpr (ROWS == 1) {
         if (first >= end) return;
         float P[16], Q[16];
         load_chunk<kForward>(L, r, first, kb, 0, vec, P);
@@ -172,8 +172,7 @@ __device__ void panel_update(double* Y, const float* L, int r, int kb, int first
 #pragma unroll
             for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
         }
-        return;
-    }
+    } else {
     for (int i0 = first; i0 < end; i0 += 2 * stride) {
         const int i1 = i0 + stride;
         const bool two = i1 < end;
@@ -209,6 +208,7 @@ __device__ void panel_update(double* Y, const float* L, int r, int kb, int first
             if (two) Y[i1 * NC + q] = acc1[q];
         }
     }
+    }
 }
 
 // The same for a block of bs < 64 rows (the last one), one entry at a time.
@@ -226,6 +226,46 @@ __device__ void panel_update_short(double* Y, const float* L, int r, int kb, int
         }
 #pragma unroll
         for (int q = 0; q < NC; ++q) Y[i * NC + q] = acc[q];
+    }
+}
+
+// The 64-row diagonal block solved for the right-hand sides q0, q0 + 8, ...
+// (CPW of them) by one warp: lanes own rows kb + lane and kb + lane + 32, and
+// the columns' shuffle and FMA chains interleave, so one serial pass of 64
+// steps serves CPW columns.  kForward: L y = c; else L^T x = y.
+template <int NC, int CPW, bool kForward>
+__device__ __forceinline__ void diag_solve(double* Y, const float* Ld, const double* rinv, int kb, int bs, int q0,
+                                           int lane) {
+    double y0[CPW], y1[CPW];
+#pragma unroll
+    for (int c = 0; c < CPW; ++c) {
+        const int q = q0 + 8 * c;
+        y0[c] = (q < NC && lane < bs) ? Y[(kb + lane) * NC + q] : 0.0;
+        y1[c] = (q < NC && lane + 32 < bs) ? Y[(kb + lane + 32) * NC + q] : 0.0;
+    }
+    for (int s = 0; s < bs; ++s) {
+        const int i = kForward ? s : bs - 1 - s;
+        const double ri = rinv[i];
+        const float l0 = kForward ? Ld[lane * (kTB + 1) + i] : Ld[i * (kTB + 1) + lane];
+        const float l1 = kForward ? Ld[(lane + 32) * (kTB + 1) + i] : Ld[i * (kTB + 1) + lane + 32];
+        const bool u0 = kForward ? lane > i : lane < i, u1 = kForward ? lane + 32 > i : lane + 32 < i;
+#pragma unroll
+        for (int c = 0; c < CPW; ++c) {
+            const double own = (i < 32) ? y0[c] : y1[c];
+            const double yi = __shfl_sync(0xffffffffu, own * ri, i & 31);
+            if (lane == (i & 31)) {
+                if (i < 32) y0[c] = yi;
+                else y1[c] = yi;
+            }
+            if (u0) y0[c] -= (double)l0 * yi;
+            if (u1) y1[c] -= (double)l1 * yi;
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < CPW; ++c) {
+        const int q = q0 + 8 * c;
+        if (q < NC && lane < bs) Y[(kb + lane) * NC + q] = y0[c];
+        if (q < NC && lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1[c];
     }
 }
 
@@ -249,6 +289,10 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
     float* Wu = W + (size_t)u * r * wcols;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool rows16 = (r & 3) == 0;  // rows of L start on 16-byte boundaries
+    // right-hand sides per solving warp; more than 8 columns a block only for a single
+    // diagonal block (r <= 64: no trailing panels, checked by the launcher)
+    constexpr int kCpw = (NC + 7) / 8;
+    static_assert(NC <= 8 || NC % 8 == 0, "columns split evenly over the 8 warps");
 
     for (int e = tid; e < NC * k; e += kTrsmThreads) {
         const int q = e / k, a = e - q * k;
@@ -270,63 +314,94 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* __restr
     for (int kb = 0; kb < k; kb += kTB) {
         const int bs = min(kTB, k - kb);
         stage_diag(kb, bs);
-        if (warp < NC) {
-            const int q = warp;
-            double y0 = lane < bs ? Y[(kb + lane) * NC + q] : 0.0;
-            double y1 = lane + 32 < bs ? Y[(kb + lane + 32) * NC + q] : 0.0;
-            for (int i = 0; i < bs; ++i) {
-                const double own = (i < 32) ? y0 : y1;
-                const double yi = __shfl_sync(0xffffffffu, own * rinv[i], i & 31);
-                if (lane == (i & 31)) {
-                    if (i < 32) y0 = yi;
-                    else y1 = yi;
-                }
-                if (lane > i) y0 -= (double)Ld[lane * (kTB + 1) + i] * yi;
-                if (lane + 32 > i) y1 -= (double)Ld[(lane + 32) * (kTB + 1) + i] * yi;
-            }
-            if (lane < bs) Y[(kb + lane) * NC + q] = y0;
-            if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
-        }
+        if (warp < (NC < 8 ? NC : 8)) diag_solve<NC, kCpw, true>(Y, Ld, rinv, kb, bs, warp, lane);
         __syncthreads();
         // every later row i: Y_i -= L[i, kb .. kb + bs) Y[kb .. kb + bs)
-        if (bs == kTB)
-            panel_update<NC, true, ROWS>(Y, L, r, kb, kb + bs + tid, k, kTrsmThreads, rows16);
-        else
-            panel_update_short<NC, true>(Y, L, r, kb, bs, kb + bs + tid, k, kTrsmThreads);
+        if constexpr (NC <= 8) {
+            if (bs == kTB)
+                panel_update<NC, true, ROWS>(Y, L, r, kb, kb + bs + tid, k, kTrsmThreads, rows16);
+            else
+                panel_update_short<NC, true>(Y, L, r, kb, bs, kb + bs + tid, k, kTrsmThreads);
+        }
     }
 
     // ---- backward: L^T x = y
     for (int kb = (k - 1) / kTB * kTB; k > 0 && kb >= 0; kb -= kTB) {
         const int bs = min(kTB, k - kb);
         stage_diag(kb, bs);
-        if (warp < NC) {
-            const int q = warp;
-            double y0 = lane < bs ? Y[(kb + lane) * NC + q] : 0.0;
-            double y1 = lane + 32 < bs ? Y[(kb + lane + 32) * NC + q] : 0.0;
-            for (int i = bs - 1; i >= 0; --i) {
-                const double own = (i < 32) ? y0 : y1;
-                const double xi = __shfl_sync(0xffffffffu, own * rinv[i], i & 31);
-                if (lane == (i & 31)) {
-                    if (i < 32) y0 = xi;
-                    else y1 = xi;
-                }
-                if (lane < i) y0 -= (double)Ld[i * (kTB + 1) + lane] * xi;
-                if (lane + 32 < i) y1 -= (double)Ld[i * (kTB + 1) + lane + 32] * xi;
-            }
-            if (lane < bs) Y[(kb + lane) * NC + q] = y0;
-            if (lane + 32 < bs) Y[(kb + lane + 32) * NC + q] = y1;
-        }
+        if (warp < (NC < 8 ? NC : 8)) diag_solve<NC, kCpw, false>(Y, Ld, rinv, kb, bs, warp, lane);
         __syncthreads();
         // every earlier row i: Y_i -= L[kb .. kb + bs, i]^T Y[kb .. kb + bs) (loads coalesced across i)
-        if (bs == kTB)
-            panel_update<NC, false, ROWS>(Y, L, r, kb, tid, kb, kTrsmThreads, false);
-        else
-            panel_update_short<NC, false>(Y, L, r, kb, bs, tid, kb, kTrsmThreads);
+        if constexpr (NC <= 8) {
+            if (bs == kTB)
+                panel_update<NC, false, ROWS>(Y, L, r, kb, tid, kb, kTrsmThreads, false);
+            else
+                panel_update_short<NC, false>(Y, L, r, kb, bs, tid, kb, kTrsmThreads);
+        }
     }
     __syncthreads();
     for (int e = tid; e < r * nc; e += kTrsmThreads) {
         const int a = e / nc, q = e - a * nc;
         Wu[(size_t)a * wcols + c0 + q] = a < k ? (float)Y[a * NC + q] : 0.f;
+    }
+}
+
+// W = L^-T (L^-1 C1) for a coreset of at most 64 rows (one diagonal block),
+// one block per unit and one thread per right-hand side: thread q substitutes
+// column q row by row (L read from shared memory as a broadcast, the columns
+// interleaved in shared memory so a warp's reads are contiguous), so no lane
+// idles on a triangular mask and no shuffle chain serialises the columns.
+constexpr int kSmallR = 64;
+__global__ void trsm_small_kernel(const float* __restrict__ Lg, const int32_t* __restrict__ rank,
+                                  const double* __restrict__ Ct, float* W, int r, int dv, int* status) {
+    __shared__ float Ls[kSmallR][kSmallR + 1];
+    __shared__ double rinv[kSmallR];
+    extern __shared__ double Ys[];                          // [k][wcols]
+    const int u = blockIdx.x, wcols = dv + 1, tid = threadIdx.x;
+    int k = rank[u];
+    if (!in_bounds(k >= 0 && k <= r && r <= kSmallR, status)) k = 0;
+    const float* L = Lg + (size_t)u * r * r;
+    const double* C = Ct + (size_t)u * wcols * r;
+    for (int e = tid; e < k * k; e += blockDim.x) {
+        const int i = e / k, j = e - i * k;
+        Ls[i][j] = j <= i ? L[(size_t)i * r + j] : 0.f;
+    }
+    for (int i = tid; i < k; i += blockDim.x) rinv[i] = 1.0 / (double)L[(size_t)i * r + i];
+    for (int e = tid; e < k * wcols; e += blockDim.x) {
+        const int q = e / k, a = e - q * k;
+        Ys[a * wcols + q] = C[(size_t)q * r + a];
+    }
+    __syncthreads();
+    if (tid < wcols) {
+        const int q = tid;
+        // forward: L y = c
+        for (int i = 0; i < k; ++i) {
+            double a0 = Ys[i * wcols + q], a1 = 0.0;
+            int j = 0;
+            for (; j + 1 < i; j += 2) {
+                a0 = fma(-(double)Ls[i][j], Ys[j * wcols + q], a0);
+                a1 = fma(-(double)Ls[i][j + 1], Ys[(j + 1) * wcols + q], a1);
+            }
+            if (j < i) a0 = fma(-(double)Ls[i][j], Ys[j * wcols + q], a0);
+            Ys[i * wcols + q] = (a0 + a1) * rinv[i];
+        }
+        // backward: L^T x = y
+        for (int i = k - 1; i >= 0; --i) {
+            double a0 = Ys[i * wcols + q], a1 = 0.0;
+            int j = i + 1;
+            for (; j + 1 < k; j += 2) {
+                a0 = fma(-(double)Ls[j][i], Ys[j * wcols + q], a0);
+                a1 = fma(-(double)Ls[j + 1][i], Ys[(j + 1) * wcols + q], a1);
+            }
+            if (j < k) a0 = fma(-(double)Ls[j][i], Ys[j * wcols + q], a0);
+            Ys[i * wcols + q] = (a0 + a1) * rinv[i];
+        }
+    }
+    __syncthreads();
+    float* Wu = W + (size_t)u * r * wcols;
+    for (int e = tid; e < r * wcols; e += blockDim.x) {
+        const int a = e / wcols;
+        Wu[e] = a < k ? (float)Ys[e] : 0.f;
     }
 }
 
@@ -419,6 +494,15 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
         if (!smem_ok(nc)) continue;
         best = nc;
         if ((long)s.units * ((s.dv + nc) / nc) * 2 >= (long)nsm * (s.r >= 1024 ? 1 : 2)) break;
+    }
+    // a single diagonal block (r <= 64): one block per unit, one thread per right-hand side
+    if (s.r <= kSmallR) {
+        const size_t smem = sizeof(double) * (size_t)s.r * (s.dv + 1);   // 132 KB at most (r = 64, dv = 256)
+        if (cudaFuncSetAttribute(trsm_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return WC_ERR_CUDA;
+        trsm_small_kernel<<<s.units, (s.dv + 1 + 31) / 32 * 32, smem, st>>>(Lg, rank, Ct, W, s.r, s.dv, status);
+        return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
     }
     if (best == 8) return launch_trsm_t<8>(s, Lg, rank, Ct, W, status, st);
     if (best == 4) return launch_trsm_t<4>(s, Lg, rank, Ct, W, status, st);
