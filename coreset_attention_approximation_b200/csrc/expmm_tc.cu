@@ -1098,10 +1098,22 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
     }
 }
 
-// V (bf16) -> fp16 copy for the value operand of the weights GEMM.
+// V (bf16) -> fp16 copy for the value operand of the weights GEMM, 8 elements
+// (16 bytes each way) a thread and iteration; count is a multiple of 8 (dv is).
 __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, size_t count) {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
-        dst[i] = __float2half_rn(__bfloat162float(src[i]));
+    const uint4* s8 = reinterpret_cast<const uint4*>(src);
+    uint4* d8 = reinterpret_cast<uint4*>(dst);
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count / 8; i += (size_t)gridDim.x * blockDim.x) {
+        const uint4 v = s8[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const __half2 h = __floats2half2_rn(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+            o[k] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        d8[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
 }
 
 // The attention's weights as the tensor cores take them: per unit and value

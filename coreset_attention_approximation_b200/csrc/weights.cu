@@ -23,8 +23,10 @@ namespace {
 template <typename T>
 __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict__ piv,
                               const float* __restrict__ F, const int32_t* __restrict__ rank, T* Ks,
-                              float* Lg, int n, int d, int r, int64_t ldf, int bins, int* status) {
-    const int a = blockIdx.x, u = blockIdx.y;
+                              float* Lg, int n, int d, int r, int64_t ldf, int bins, int tpr, int* status) {
+    // tpr threads a row, blockDim.x / tpr rows a block
+    const int a = blockIdx.x * (blockDim.x / tpr) + threadIdx.x / tpr, u = blockIdx.y, t = threadIdx.x % tpr;
+    if (a >= r) return;
     int k = rank[u];
     if (!in_bounds(k >= 0 && k <= r, status)) k = 0;
     const int base = (u % bins) * n;  // the bin's first key within the caller's unit
@@ -33,12 +35,10 @@ __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict
     if (!in_bounds(a >= k || (p >= 0 && p < n), status)) p = -1;
     if (!in_bounds(pk < n && (pk >= 0 || a >= k), status)) pk = -1;
     T* ks = Ks + ((size_t)u * r + a) * d;
-    for (int c = threadIdx.x; c < d; c += blockDim.x)
-        ks[c] = pk >= 0 ? K[((size_t)u * n + pk) * d + c] : T(0.f);
+    for (int c = t; c < d; c += tpr) ks[c] = pk >= 0 ? K[((size_t)u * n + pk) * d + c] : T(0.f);
     float* lrow = Lg + ((size_t)u * r + a) * r;
     const float* Fu = F + (size_t)u * r * ldf;
-    for (int b = threadIdx.x; b < r; b += blockDim.x)
-        lrow[b] = (p >= 0 && b <= a) ? Fu[(int64_t)b * ldf + p] : 0.f;
+    for (int b = t; b < r; b += tpr) lrow[b] = (p >= 0 && b <= a) ? Fu[(int64_t)b * ldf + p] : 0.f;
 }
 
 // C1 from the partial sums of the key splits, in fp64:
@@ -50,8 +50,10 @@ __global__ void gather_kernel(const T* __restrict__ K, const int32_t* __restrict
 __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t* __restrict__ rank, double* Ct,
                                 int nsplit, int r, int dv, const int32_t* __restrict__ piv,
                                 const double* __restrict__ cdot, const double* __restrict__ kk, int bins, int n_all,
-                                double beta, const double* __restrict__ shift, int* status) {
-    const int a = blockIdx.x, u = blockIdx.y;
+                                double beta, const double* __restrict__ shift, int tpr, int* status) {
+    // tpr threads a coreset row, blockDim.x / tpr rows a block
+    const int a = blockIdx.x * (blockDim.x / tpr) + threadIdx.x / tpr, u = blockIdx.y, t = threadIdx.x % tpr;
+    if (a >= r) return;
     if (a >= rank[u] || !in_bounds(rank[u] <= r, status)) return;
     double rho = -shift[u];
     if (cdot) {
@@ -64,7 +66,7 @@ __global__ void merge_c1_kernel(const float* __restrict__ c1part, const int32_t*
     const float* part = c1part + (size_t)u * nsplit * r * w;
     double mx = -INFINITY;
     for (int sp = 0; sp < nsplit; ++sp) mx = fmax(mx, (double)part[((size_t)sp * r + a) * w + dv + 1]);
-    for (int c = threadIdx.x; c < wcols; c += blockDim.x) {
+    for (int c = t; c < wcols; c += tpr) {
         double acc = 0.0;
         if (mx > -INFINITY) {
             for (int sp = 0; sp < nsplit; ++sp) {
@@ -429,15 +431,21 @@ wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const
     const WsLayout L = make_layout(s);
     float* Lg = reinterpret_cast<float*>(ws + L.lg);
     int* status = reinterpret_cast<int*>(ws + L.status);
-    dim3 grid(s.r, s.units);
+    // a row's copies take max(d, r) elements: give it that many threads (whole warps, at most
+    // 256) and put several short rows in a block (many tiny blocks leave the GPU's block
+    // scheduler the bottleneck)
+    const int w = s.d > s.r ? s.d : s.r;
+    const int tpr = w >= 256 ? 256 : (w + 31) / 32 * 32;
+    const int rpb = 256 / tpr;
+    dim3 grid((s.r + rpb - 1) / rpb, s.units);
     if (s.dtype == WC_BF16)
-        gather_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(K), piv, F, rank,
-                                                           static_cast<__nv_bfloat16*>(Ks), Lg, s.n, s.d, s.r,
-                                                           s.ldf, s.bins, status);
+        gather_kernel<__nv_bfloat16><<<grid, rpb * tpr, 0, st>>>(static_cast<const __nv_bfloat16*>(K), piv, F, rank,
+                                                                 static_cast<__nv_bfloat16*>(Ks), Lg, s.n, s.d, s.r,
+                                                                 s.ldf, s.bins, tpr, status);
     else
-        gather_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(K), piv, F, rank,
-                                                   static_cast<float*>(Ks), Lg, s.n, s.d, s.r, s.ldf, s.bins,
-                                                   status);
+        gather_kernel<float><<<grid, rpb * tpr, 0, st>>>(static_cast<const float*>(K), piv, F, rank,
+                                                         static_cast<float*>(Ks), Lg, s.n, s.d, s.r, s.ldf, s.bins,
+                                                         tpr, status);
     return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -470,11 +478,12 @@ wc_status launch_solve(const Shape& s, const int32_t* piv, const int32_t* rank, 
     const WsLayout L = make_layout(s);
     double* Ct = reinterpret_cast<double*>(ws + L.y);
     int* status = reinterpret_cast<int*>(ws + L.status);
-    merge_c1_kernel<<<dim3(s.r, s.units), 160, 0, st>>>(
+    // a warp per coreset row, 8 rows a block
+    merge_c1_kernel<<<dim3((s.r + 7) / 8, s.units), 256, 0, st>>>(
         reinterpret_cast<const float*>(ws + L.c1part), rank, Ct, s.nsplit, s.r, s.dv, piv,
         s.center ? reinterpret_cast<const double*>(ws + L.cdot) : nullptr,
         s.center ? reinterpret_cast<const double*>(ws + L.kk) : nullptr, s.bins, s.n_all, s.beta,
-        reinterpret_cast<const double*>(ws + L.shift), status);
+        reinterpret_cast<const double*>(ws + L.shift), 32, status);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
     // right-hand sides per block: 8 (the fewest re-reads of L, and each block
     // repeats the serial diagonal solves), fewer only while the blocks would
