@@ -30,6 +30,12 @@
 // Blocks of one unit wait on each other, so a wave with C > 1 is launched
 // cooperatively (all blocks co-resident); every wait gives up after the
 // shape's timeout and records WC_ERR_TIMEOUT.
+//
+// Few short units (all of them on the GPU at once, each unit's keys and factor
+// within the shared memory of a cluster of up to 8 blocks) take the resident
+// variant below instead: the same steps on shared-memory copies, the blocks
+// meeting at the cluster barrier.
+#include <cooperative_groups.h>
 #include <type_traits>
 
 #include "wc_common.cuh"
@@ -229,6 +235,66 @@ __device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, 
         cor[0] += (double)a0;
         cor[1] += (double)a1;
     }
+}
+
+// One row's <k_i, k_s> and correction, from shared memory (the resident
+// variant with a row per thread): the same sums, in the same order, as the
+// two-row forms above.
+__device__ __forceinline__ double key_dot1(const __nv_bfloat16* Kt, int m, int d, const float* ksf) {
+    double dot = 0.0;
+#pragma unroll 4
+    for (int c0 = 0; c0 < d; c0 += 8) {
+        const float4 k0 = *reinterpret_cast<const float4*>(ksf + c0);
+        const float4 k1 = *reinterpret_cast<const float4*>(ksf + c0 + 4);
+        const float kc[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+        float a0 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t w = (uint32_t)*reinterpret_cast<const unsigned short*>(Kt + (size_t)(c0 + c) * m) << 16;
+            a0 = fmaf(__uint_as_float(w), kc[c], a0);
+        }
+        dot += (double)a0;
+    }
+    return dot;
+}
+
+__device__ __forceinline__ double key_dot1(const float* Kt, int m, int d, const double* ks) {
+    double dot = 0.0;
+#pragma unroll 8
+    for (int c = 0; c < d; ++c) dot += (double)Kt[(size_t)c * m] * ks[c];
+    return dot;
+}
+
+__device__ __forceinline__ double correction1(const float* Fi, int m, int j, const float* fs) {
+    double cor = 0.0;
+    int c0 = 0;
+    for (; c0 + 32 <= j; c0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = Fi[(size_t)(c0 + c) * m];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 f0 = *reinterpret_cast<const float4*>(fs + c0 + 8 * q);
+            const float4 f1 = *reinterpret_cast<const float4*>(fs + c0 + 8 * q + 4);
+            const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            float a0 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a0 = fmaf(v[8 * q + c], f[c], a0);
+            cor += (double)a0;
+        }
+    }
+    for (; c0 + 8 <= j; c0 += 8) {
+        float a0 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) a0 = fmaf(Fi[(size_t)(c0 + c) * m], fs[c0 + c], a0);
+        cor += (double)a0;
+    }
+    if (c0 < j) {
+        float a0 = 0.f;
+        for (int c = c0; c < j; ++c) a0 = fmaf(Fi[(size_t)c * m], fs[c], a0);
+        cor += (double)a0;
+    }
+    return cor;
 }
 
 // T: element type of K; TK: of the transposed copy that every step streams
@@ -498,6 +564,294 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
     }
 }
 
+// ---- resident variant: a unit's keys and factor held in shared memory ----
+//
+// When a unit's transposed keys and factor columns fit in the shared memory of
+// a cluster of at most kMaxCluster blocks (short heads: n r fp32 plus n d key
+// elements) and all units fit on the GPU at once (few units: the factor in
+// shared memory allows far fewer units at a time than streaming it), each block
+// keeps its slice of Kt and of F for the whole run: a step reads no global
+// memory but the pivot's key when centred, writes none (F and the pivots go
+// out after the last step), and the unit's blocks meet at the cluster barrier,
+// the slice sums, the pivot, its key and its factor row travelling through
+// distributed shared memory.  Every row's arithmetic is that of
+// rpcholesky_kernel (same dot and correction order, same scans and draw), so
+// results agree with it wherever the slice boundaries do.
+constexpr int kMaxCluster = 8;
+// threads per resident block, a row each per pass (measured against 256
+// threads with two rows each: about 5 % faster on one 512-key unit)
+constexpr int kResThreads = 512;
+
+struct PivMsg {
+    double d_s;
+    int s, stop;
+};
+
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) / 16 * 16; }
+
+// Shared-memory plan of a resident block: m rows, r pivots, d dims, key copy
+// elements of tk bytes.  Offsets in the order the kernel carves them.
+struct ResidentSmem {
+    size_t dg, scan, bsum, bmax, uj, ks, ksf, fs, msg, pv, f, kt, ispiv, total;
+    __host__ __device__ ResidentSmem(int m, int r, int d, int tk, int nt) {
+        size_t o = 0;
+        dg = o;    o = align16(o + (size_t)m * 8);
+        scan = o;  o = align16(o + (size_t)nt * 8);
+        bsum = o;  o = align16(o + (size_t)kMaxCluster * 8);
+        bmax = o;  o = align16(o + (size_t)kMaxCluster * 8);
+        uj = o;    o = align16(o + (size_t)r * 8);
+        ks = o;    o = align16(o + (size_t)d * 8);
+        ksf = o;   o = align16(o + (size_t)d * 4);
+        fs = o;    o = align16(o + (size_t)r * 4);
+        msg = o;   o = align16(o + sizeof(PivMsg));
+        pv = o;    o = align16(o + (size_t)r * 4);
+        f = o;     o = align16(o + (size_t)r * m * 4);
+        kt = o;    o = align16(o + (size_t)d * m * tk);
+        ispiv = o; o = align16(o + (size_t)m);
+        total = o;
+    }
+};
+
+namespace cg = cooperative_groups;
+
+template <typename T, typename TK, int NT>
+__global__ void __launch_bounds__(NT, 1) rpcholesky_resident_kernel(const SelectArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int CL = (int)cluster.num_blocks();
+    const int blk = (int)cluster.block_rank();
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int unit = blockIdx.x / CL;
+    const int n = a.n, d = a.d, r = a.r, m = a.m;
+    const int64_t ldf = a.ldf;
+    const int r0 = min(n, blk * m);
+    const int r1 = min(n, r0 + m);
+    const int mlen = r1 - r0;
+    // rows this block writes to F: its slice, and for the last block the
+    // padding up to ldf (F is zero there); m is a multiple of 64 and at least
+    // ldf - r0 for the last block
+    const int64_t tail = ldf - r0;
+    const int rows = tail < m ? (tail > 0 ? (int)tail : 0) : m;
+
+    const ResidentSmem L(m, r, d, (int)sizeof(TK), NT);
+    double* dg = reinterpret_cast<double*>(smem + L.dg);
+    double* scan = reinterpret_cast<double*>(smem + L.scan);
+    double* bsum = reinterpret_cast<double*>(smem + L.bsum);
+    double* bmax = reinterpret_cast<double*>(smem + L.bmax);
+    double* uj = reinterpret_cast<double*>(smem + L.uj);
+    double* ks = reinterpret_cast<double*>(smem + L.ks);
+    float* ksf = reinterpret_cast<float*>(smem + L.ksf);
+    float* fs = reinterpret_cast<float*>(smem + L.fs);
+    PivMsg* msg = reinterpret_cast<PivMsg*>(smem + L.msg);
+    int* pv = reinterpret_cast<int*>(smem + L.pv);     // the pivots, written out at the end
+    float* Fs = reinterpret_cast<float*>(smem + L.f);   // [r][m]
+    TK* Kts = reinterpret_cast<TK*>(smem + L.kt);      // [d][m]
+    unsigned char* ispiv = smem + L.ispiv;
+    __shared__ unsigned long long lmax_bits;
+
+    const T* K = static_cast<const T*>(a.K) + (size_t)unit * n * d;
+    const double* kb = a.kbar ? a.kbar + (size_t)(unit / a.bins) * d : nullptr;
+    float* F = a.F + (size_t)unit * r * ldf;
+    int* status = a.status;
+
+    // ---- the unit's pivot draws (they depend on nothing the steps compute);
+    // the slice's keys, transposed into shared memory; beta |k_i|^2
+    for (int jj = tid; jj < r; jj += NT) uj[jj] = pivot_uniform(a.seed, (uint32_t)jj, a.unit_base + (uint32_t)unit);
+    if (tid == 0) lmax_bits = 0ull;
+    __syncthreads();
+    double lmax = 0.0;
+    for (int il = tid; il < m; il += NT) {
+        double v = 0.0;
+        if (il < mlen) {
+            const T* krow = K + (size_t)(r0 + il) * d;
+            double ss = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const T kv = krow[c];
+                double x = (double)to_f32(kv);
+                if (kb) x -= kb[c];
+                ss += x * x;
+                if constexpr (std::is_same<T, TK>::value) Kts[(size_t)c * m + il] = kb ? TK((float)x) : kv;
+                else Kts[(size_t)c * m + il] = (TK)(float)x;
+            }
+            v = a.beta * ss;
+        } else {
+            for (int c = 0; c < d; ++c) Kts[(size_t)c * m + il] = TK(0.f);
+        }
+        dg[il] = v;
+        ispiv[il] = 0;
+        lmax = fmax(lmax, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if (lane == 0 && lmax > 0.0) atomicMax(&lmax_bits, (unsigned long long)__double_as_longlong(lmax));
+    __syncthreads();
+    if (tid < CL) cluster.map_shared_rank(bmax, tid)[blk] = __longlong_as_double((long long)lmax_bits);
+    cluster.sync();
+    double shift = 0.0;
+    for (int c = 0; c < CL; ++c) shift = fmax(shift, bmax[c]);
+    bool alive = isfinite(shift);
+    if (!alive && blk == 0 && tid == 0) record_status(status, WC_ERR_NUMERIC);
+    const double hmax = 1.0;  // the shifted diagonal's maximum
+
+    if (alive) {
+        for (int il = tid; il < mlen; il += NT) dg[il] = exp(dg[il] - shift);
+        __syncthreads();
+        int lo, hi;
+        chunk_of<NT>(tid, mlen, &lo, &hi);
+        double sum = 0.0;
+        for (int il = lo; il < hi; ++il) sum += dg[il];
+        const double tot = block_scan<NT>(sum, scan);
+        if (tid < CL) cluster.map_shared_rank(bsum, tid)[blk] = tot;
+        cluster.sync();
+    }
+
+    int final_rank = alive ? r : 0;
+    for (int j = 0; alive && j < r; ++j) {
+        // 1. the block whose slice holds t = u_j * sum(d), from the slice sums:
+        // every thread of every block of the unit takes the same decision
+        double total = 0.0;
+        for (int c = 0; c < CL; ++c) total += bsum[c];
+        if (!(total > 0.0)) {
+            if (isnan(total) && blk == 0 && tid == 0) record_status(status, WC_ERR_NUMERIC);
+            final_rank = j;
+            break;
+        }
+        const double tau = uj[j] * total;
+        int owner = -1;
+        double base = 0.0;
+        {
+            double run = 0.0;
+            for (int c = 0; c < CL; ++c) {
+                const double nxt = run + bsum[c];
+                if (nxt > tau) { owner = c; base = run; break; }
+                run = nxt;
+            }
+            if (owner < 0) {  // rounding left tau at the top: last block with mass
+                run = 0.0;
+                for (int c = 0; c < CL; ++c) {
+                    const double p = bsum[c];
+                    if (p > 0.0) { owner = c; base = run; }
+                    run += p;
+                }
+            }
+        }
+
+        // 2. in the owner, the first thread whose inclusive slice prefix passes
+        // tau (prefixes of non-negative terms do not decrease), else the last
+        // thread, scans its chunk; its warp sends the pivot, its key and its
+        // factor row to every block of the unit
+        if (blk == owner) {
+            const bool past = base + scan[tid] > tau;
+            const bool prev = tid > 0 && base + scan[tid - 1] > tau;
+            const bool mine = (past && !prev) || (tid == NT - 1 && !past);
+            const unsigned bal = __ballot_sync(0xffffffffu, mine);
+            if (bal) {
+                int sl = -1, stop = 1;
+                double ds = 0.0;
+                if (mine) {
+                    int lo, hi;
+                    chunk_of<NT>(tid, mlen, &lo, &hi);
+                    double run = tid == 0 ? base : base + scan[tid - 1];
+                    for (int il = lo; il < hi; ++il) {
+                        run += dg[il];
+                        if (run > tau) { sl = il; break; }
+                    }
+                    if (sl < 0) {  // rounding: last positive entry of the chunk, else of the slice
+                        for (int il = hi - 1; il >= lo && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                        for (int il = mlen - 1; il >= 0 && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                    }
+                    ds = sl >= 0 ? dg[sl] : 0.0;
+                    stop = !(ds > a.eps * hmax);
+                }
+                const int src = __ffs(bal) - 1;
+                sl = __shfl_sync(0xffffffffu, sl, src);
+                stop = __shfl_sync(0xffffffffu, stop, src);
+                ds = __shfl_sync(0xffffffffu, ds, src);
+                for (int p = 0; p < CL; ++p) {
+                    if (sl >= 0) {
+                        double* ksp = cluster.map_shared_rank(ks, p);
+                        float* ksfp = cluster.map_shared_rank(ksf, p);
+                        float* fsp = cluster.map_shared_rank(fs, p);
+                        for (int c = lane; c < d; c += 32) {
+                            const double kv = kb ? (double)to_f32(K[(size_t)(r0 + sl) * d + c]) - kb[c]
+                                                 : (double)to_f32(Kts[(size_t)c * m + sl]);
+                            ksp[c] = kv;
+                            ksfp[c] = (float)kv;
+                        }
+                        for (int c = lane; c < j; c += 32) fsp[c] = Fs[(size_t)c * m + sl];
+                    }
+                    if (lane == 0) {
+                        PivMsg* mp = cluster.map_shared_rank(msg, p);
+                        mp->s = r0 + sl;
+                        mp->d_s = ds;
+                        mp->stop = stop;
+                    }
+                }
+            }
+        }
+        cluster.sync();
+        if (msg->stop) { final_rank = j; break; }
+        const int s = msg->s;
+        const double ds = msg->d_s;
+        if (!in_bounds(s >= 0 && s < n, status)) {  // every block reads the same s: all stop here
+            final_rank = j;
+            break;
+        }
+        if (tid == 0) pv[j] = s;
+
+        // 3. column j over this block's rows, and the residual downdate (the
+        // pivot's own row leaves the residual here); the factor goes out to
+        // global memory after the last step, so that no step's barrier waits
+        // for global stores
+        const double root = sqrt(ds);
+        const int spl = s - r0;
+        float* Fsj = Fs + (size_t)j * m;
+        for (int il = tid; il < rows; il += NT) {
+            double dot;
+            if constexpr (std::is_same<TK, float>::value) dot = key_dot1(Kts + il, m, d, ks);
+            else dot = key_dot1(Kts + il, m, d, ksf);
+            const double cor = correction1(Fs + il, m, j, fs);
+            double f = 0.0;
+            if (il < mlen && !ispiv[il]) f = (exp(a.beta * dot - shift) - cor) / root;
+            Fsj[il] = (float)f;
+            if (il < mlen) {
+                const double nd = dg[il] - f * f;
+                dg[il] = il == spl ? 0.0 : (nd > 0.0 ? nd : 0.0);
+                if (il == spl) ispiv[il] = 1;
+            }
+        }
+        __syncthreads();
+
+        // 4. new slice sum to every block, then close the step
+        {
+            int lo, hi;
+            chunk_of<NT>(tid, mlen, &lo, &hi);
+            double sum = 0.0;
+            for (int il = lo; il < hi; ++il) sum += dg[il];
+            const double tot = block_scan<NT>(sum, scan);
+            if (tid < CL) cluster.map_shared_rank(bsum, tid)[blk] = tot;
+        }
+        cluster.sync();
+    }
+
+    // ---- the factor's columns (zero from the rank on) and the pivots (-1 from
+    // the rank on) out to global memory
+    __syncthreads();
+    for (int jj = 0; jj < r; ++jj) {
+        float* Fj = F + (int64_t)jj * ldf + r0;
+        const float* Fsj = Fs + (size_t)jj * m;
+        for (int g = tid; g < rows / 2; g += NT)
+            *reinterpret_cast<float2*>(Fj + 2 * g) =
+                jj < final_rank ? *reinterpret_cast<const float2*>(Fsj + 2 * g) : make_float2(0.f, 0.f);
+    }
+    if (blk == 0) {
+        const int off = (unit % a.bins) * a.bin_keys;
+        for (int jj = tid; jj < r; jj += NT) a.piv[(size_t)unit * r + jj] = jj < final_rank ? pv[jj] + off : -1;
+        if (tid == 0) a.rank[unit] = final_rank;
+    }
+    cluster.sync();  // no block leaves while a peer may still write to its shared memory
+}
+
 struct SelectPlan {
     int C = 0, m = 0;   // blocks per unit, rows per block
     long cap = 0;       // blocks the GPU holds at once with m rows each
@@ -573,6 +927,71 @@ wc_status run_select(const Shape& s, const SelectPlan& p, SelectArgs a, char* ws
     return WC_OK;
 }
 
+// Cluster size and rows per block of the resident variant, or false where a
+// unit does not fit in the shared memory of kMaxCluster blocks or the units
+// do not all fit on the GPU at once.  The fewest blocks per unit that hold
+// it, doubled while the launch would leave more than half of the SMs idle and
+// blocks keep at least 128 rows.
+template <typename T, typename TK, int NT>
+bool plan_resident(const Shape& s, int nsm, int max_smem, int* cl_out, int* m_out, size_t* smem_out) {
+    auto rows_for = [&](int cl) { return ((s.n + cl - 1) / cl + 63) / 64 * 64; };
+    const size_t avail = (size_t)max_smem - 1024;
+    int cl = 1;
+    while (cl <= kMaxCluster && ResidentSmem(rows_for(cl), s.r, s.d, (int)sizeof(TK), NT).total > avail) cl *= 2;
+    if (cl > kMaxCluster) return false;
+    while (cl < kMaxCluster && (long)s.units * cl * 2 <= nsm && (s.n + 2 * cl - 1) / (2 * cl) >= 128) cl *= 2;
+    const int m = rows_for(cl);
+    if ((long)(cl - 1) * m >= s.n) return false;  // every block of a unit holds rows
+    const size_t smem = ResidentSmem(m, s.r, s.d, (int)sizeof(TK), NT).total;
+    auto kern = rpcholesky_resident_kernel<T, TK, NT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(s.units * cl));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+        cudaGetLastError();
+        return false;
+    }
+    // A resident unit holds its whole factor in shared memory, so far fewer
+    // units run at once than in the streaming kernel (ViT-sized heads: about 80
+    // against about 300).  Its step is shorter, which pays only while every
+    // unit runs at once.
+    if (s.units > clusters) return false;
+    *cl_out = cl;
+    *m_out = m;
+    *smem_out = smem;
+    return true;
+}
+
+template <typename T, typename TK, int NT>
+wc_status run_resident(const Shape& s, int cl, size_t smem, const SelectArgs& a, cudaStream_t st) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(s.units * cl));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, rpcholesky_resident_kernel<T, TK, NT>, a) == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
 template <typename T, typename TK>
 wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank, char* ws,
                           cudaStream_t st) {
@@ -588,6 +1007,31 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     if ((size_t)max_smem <= fixed) return WC_ERR_UNSUPPORTED;
     int m_max = (int)(((size_t)max_smem - fixed) / 9) / kRowAlign * kRowAlign;
     m_max = m_max > (1 << 20) ? (1 << 20) : m_max;
+
+    SelectArgs a;
+    a.K = K; a.piv = piv; a.F = F; a.rank = rank;
+    a.bins = s.bins;
+    a.bin_keys = s.n;
+    a.unit_base = (uint32_t)s.unit_base * (uint32_t)s.bins;   // bin view: unit u * bins + bin
+    a.kbar = s.center ? reinterpret_cast<const double*>(ws + L.kbar) : nullptr;
+    a.Kt = ws + L.kt;
+    a.sync = reinterpret_cast<UnitSync*>(ws + L.sync);
+    a.partials = reinterpret_cast<double*>(ws + L.partials);
+    a.status = reinterpret_cast<int*>(ws + L.status);
+    a.ldf = s.ldf; a.n = s.n; a.d = s.d; a.r = s.r;
+    a.beta = s.beta; a.eps = s.eps; a.seed = s.seed; a.timeout_ns = s.timeout_ns;
+    a.unit0 = 0;
+
+    // short units: keys and factor resident in the shared memory of a cluster
+    {
+        int cl = 0, m = 0;
+        size_t smem = 0;
+        if (plan_resident<T, TK, kResThreads>(s, nsm, max_smem, &cl, &m, &smem)) {
+            a.C = cl;
+            a.m = m;
+            return run_resident<T, TK, kResThreads>(s, cl, smem, a, st);
+        }
+    }
 
     // 256-thread blocks, unless the launch is one co-resident wave either way
     // and 128-thread blocks leave the busiest SM fewer rows: with 2 blocks per
@@ -607,19 +1051,7 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     if (p.cap < 1) return WC_ERR_CUDA;
     if (p.C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
 
-    SelectArgs a;
-    a.K = K; a.piv = piv; a.F = F; a.rank = rank;
-    a.bins = s.bins;
-    a.bin_keys = s.n;
-    a.unit_base = (uint32_t)s.unit_base * (uint32_t)s.bins;   // bin view: unit u * bins + bin
-    a.kbar = s.center ? reinterpret_cast<const double*>(ws + L.kbar) : nullptr;
-    a.Kt = ws + L.kt;
-    a.sync = reinterpret_cast<UnitSync*>(ws + L.sync);
-    a.partials = reinterpret_cast<double*>(ws + L.partials);
-    a.status = reinterpret_cast<int*>(ws + L.status);
-    a.ldf = s.ldf; a.n = s.n; a.d = s.d; a.r = s.r;
     a.C = p.C; a.m = p.m;
-    a.beta = s.beta; a.eps = s.eps; a.seed = s.seed; a.timeout_ns = s.timeout_ns;
 
     if (cudaMemsetAsync(ws + L.sync, 0, sizeof(UnitSync) * (size_t)s.units, st) != cudaSuccess) return WC_ERR_CUDA;
     return use128 ? run_select<T, TK, 128>(s, p, a, ws, st) : run_select<T, TK, 256>(s, p, a, ws, st);
