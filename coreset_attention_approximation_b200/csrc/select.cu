@@ -39,6 +39,7 @@
 #include <type_traits>
 
 #include "wc_common.cuh"
+#include "wc_exp2.cuh"
 #include "wc_internal.h"
 
 namespace wc {
@@ -88,7 +89,8 @@ __host__ __device__ inline size_t select_smem_bytes(int m, int r, int d) {
            + (size_t)kThreads * 8 // per-thread inclusive scan
            + (size_t)kMaxBlocksPerUnit * 8  // the unit's block sums of a step
            + (size_t)d * 8        // pivot key
-           + (size_t)r * 4        // F[s, 0..j)
+           + (size_t)d * 8        // pivot key as fp32 pairs
+           + (size_t)r * 8        // F[s, 0..j) as pairs
            + (size_t)m            // pivot flags
            + 64;                  // broadcast scalars
 }
@@ -149,33 +151,44 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
     return v;
 }
 
+// The two-row sums below run the two rows' fp32 products as packed pairs
+// (fma.rn.f32x2: per lane the rounding of fmaf), against the pivot's values
+// held twice over in shared memory ({v, v} pairs, read four floats at a time).
+
 // <k_i, k_s> for the 2 rows at Kt + i0 (column stride ldf): products of 8
-// consecutive dimensions summed in fp32, the chunks summed in fp64.
+// consecutive dimensions summed in fp32, the chunks summed in fp64.  ks2: the
+// pivot key as fp32 pairs (exact: it holds bf16 values); ks: in fp64.
 template <typename T>
-__device__ __forceinline__ void key_dots(const T* Kt, int64_t ldf, int d, const double* ks, double dot[2]);
+__device__ __forceinline__ void key_dots(const T* Kt, int64_t ldf, int d, const float2* ks2, const double* ks,
+                                         double dot[2]);
+
+__device__ __forceinline__ float2 bf16_pair(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 
 template <>
 __device__ __forceinline__ void key_dots<__nv_bfloat16>(const __nv_bfloat16* Kt, int64_t ldf, int d,
-                                                       const double* ks, double dot[2]) {
+                                                       const float2* ks2, const double*, double dot[2]) {
     dot[0] = dot[1] = 0.0;
 #pragma unroll 4
     for (int c0 = 0; c0 < d; c0 += 8) {
-        float a0 = 0.f, a1 = 0.f;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint32_t w = ld_stream_u32(Kt + (int64_t)(c0 + c) * ldf);
-            const float kc = (float)ks[c0 + c];  // exact: ks holds bf16 values
-            a0 = fmaf(__uint_as_float(w << 16), kc, a0);
-            a1 = fmaf(__uint_as_float(w & 0xffff0000u), kc, a1);
+        for (int c = 0; c < 8; c += 2) {
+            const float4 kk = *reinterpret_cast<const float4*>(ks2 + c0 + c);
+            const uint32_t w0 = ld_stream_u32(Kt + (int64_t)(c0 + c) * ldf);
+            const uint32_t w1 = ld_stream_u32(Kt + (int64_t)(c0 + c + 1) * ldf);
+            acc = fma2(bf16_pair(w0), make_float2(kk.x, kk.y), acc);
+            acc = fma2(bf16_pair(w1), make_float2(kk.z, kk.w), acc);
         }
-        dot[0] += (double)a0;
-        dot[1] += (double)a1;
+        dot[0] += (double)acc.x;
+        dot[1] += (double)acc.y;
     }
 }
 
 template <>
-__device__ __forceinline__ void key_dots<float>(const float* Kt, int64_t ldf, int d, const double* ks,
-                                               double dot[2]) {
+__device__ __forceinline__ void key_dots<float>(const float* Kt, int64_t ldf, int d, const float2*,
+                                               const double* ks, double dot[2]) {
     // fp32 (or centred) keys: products and sums in fp64
     dot[0] = dot[1] = 0.0;
 #pragma unroll 8
@@ -187,10 +200,42 @@ __device__ __forceinline__ void key_dots<float>(const float* Kt, int64_t ldf, in
     }
 }
 
+// The same two-row dots with the keys in shared memory (column stride m).
+__device__ __forceinline__ void key_dots_shared(const __nv_bfloat16* Kt, int m, int d, const float2* ks2,
+                                                const double*, double dot[2]) {
+    dot[0] = dot[1] = 0.0;
+#pragma unroll 4
+    for (int c0 = 0; c0 < d; c0 += 8) {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const float4 kk = *reinterpret_cast<const float4*>(ks2 + c0 + c);
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(Kt + (size_t)(c0 + c) * m);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(Kt + (size_t)(c0 + c + 1) * m);
+            acc = fma2(bf16_pair(w0), make_float2(kk.x, kk.y), acc);
+            acc = fma2(bf16_pair(w1), make_float2(kk.z, kk.w), acc);
+        }
+        dot[0] += (double)acc.x;
+        dot[1] += (double)acc.y;
+    }
+}
+
+__device__ __forceinline__ void key_dots_shared(const float* Kt, int m, int d, const float2*, const double* ks,
+                                                double dot[2]) {
+    dot[0] = dot[1] = 0.0;
+#pragma unroll 8
+    for (int c = 0; c < d; ++c) {
+        const float2 v = *reinterpret_cast<const float2*>(Kt + (size_t)c * m);
+        const double kc = ks[c];
+        dot[0] += (double)v.x * kc;
+        dot[1] += (double)v.y * kc;
+    }
+}
+
 // sum_{c<j} F[c, i] F[c, s] for the 2 rows at Fi (column stride ldf): products
 // of 8 consecutive columns summed in fp32, the chunks summed in fp64.  32
-// columns are loaded before any is used.
-__device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, const float* fs, double cor[2]) {
+// columns are loaded before any is used.  fs2: F[s, c] as pairs.
+__device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, const float2* fs2, double cor[2]) {
     cor[0] = cor[1] = 0.0;
     int c0 = 0;
     for (; c0 + 32 <= j; c0 += 32) {
@@ -199,41 +244,36 @@ __device__ __forceinline__ void correction(const float* Fi, int64_t ldf, int j, 
         for (int c = 0; c < 32; ++c) v[c] = ld_stream_f2(Fi + (int64_t)(c0 + c) * ldf);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float4 f0 = *reinterpret_cast<const float4*>(fs + c0 + 8 * q);
-            const float4 f1 = *reinterpret_cast<const float4*>(fs + c0 + 8 * q + 4);
-            const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-            float a0 = 0.f, a1 = 0.f;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                a0 = fmaf(v[8 * q + c].x, f[c], a0);
-                a1 = fmaf(v[8 * q + c].y, f[c], a1);
+            for (int c = 0; c < 8; c += 2) {
+                const float4 ff = *reinterpret_cast<const float4*>(fs2 + c0 + 8 * q + c);
+                acc = fma2(v[8 * q + c], make_float2(ff.x, ff.y), acc);
+                acc = fma2(v[8 * q + c + 1], make_float2(ff.z, ff.w), acc);
             }
-            cor[0] += (double)a0;
-            cor[1] += (double)a1;
+            cor[0] += (double)acc.x;
+            cor[1] += (double)acc.y;
         }
     }
     for (; c0 + 8 <= j; c0 += 8) {
         float2 v[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) v[c] = ld_stream_f2(Fi + (int64_t)(c0 + c) * ldf);
-        float a0 = 0.f, a1 = 0.f;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            a0 = fmaf(v[c].x, fs[c0 + c], a0);
-            a1 = fmaf(v[c].y, fs[c0 + c], a1);
+        for (int c = 0; c < 8; c += 2) {
+            const float4 ff = *reinterpret_cast<const float4*>(fs2 + c0 + c);
+            acc = fma2(v[c], make_float2(ff.x, ff.y), acc);
+            acc = fma2(v[c + 1], make_float2(ff.z, ff.w), acc);
         }
-        cor[0] += (double)a0;
-        cor[1] += (double)a1;
+        cor[0] += (double)acc.x;
+        cor[1] += (double)acc.y;
     }
     if (c0 < j) {
-        float a0 = 0.f, a1 = 0.f;
-        for (int c = c0; c < j; ++c) {
-            const float2 v = ld_stream_f2(Fi + (int64_t)c * ldf);
-            a0 = fmaf(v.x, fs[c], a0);
-            a1 = fmaf(v.y, fs[c], a1);
-        }
-        cor[0] += (double)a0;
-        cor[1] += (double)a1;
+        float2 acc = make_float2(0.f, 0.f);
+        for (int c = c0; c < j; ++c) acc = fma2(ld_stream_f2(Fi + (int64_t)c * ldf), fs2[c], acc);
+        cor[0] += (double)acc.x;
+        cor[1] += (double)acc.y;
     }
 }
 
@@ -318,8 +358,9 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
     double* scan = dg + a.m;
     double* bsum = scan + kThreads;  // the scan array is planned for the larger block
     double* ks = bsum + kMaxBlocksPerUnit;
-    float* fs = reinterpret_cast<float*>(ks + d);
-    unsigned char* ispiv = reinterpret_cast<unsigned char*>(fs + r);
+    float2* ks2 = reinterpret_cast<float2*>(ks + d);
+    float2* fs2 = ks2 + d;
+    unsigned char* ispiv = reinterpret_cast<unsigned char*>(fs2 + r);
     __shared__ Bcast bc;
 
     const T* K = static_cast<const T*>(a.K) + (size_t)unit * n * d;
@@ -489,7 +530,11 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
         }
 
         // 3. pivot key and F[s, 0..j) into shared memory
-        for (int c = tid; c < d; c += NT) ks[c] = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
+        for (int c = tid; c < d; c += NT) {
+            const double kv = (double)to_f32(K[(size_t)s * d + c]) - (kb ? kb[c] : 0.0);
+            ks[c] = kv;
+            ks2[c] = make_float2((float)kv, (float)kv);
+        }
         for (int c0 = tid; c0 < j; c0 += 8 * NT) {  // 8 loads in flight before the stores
             float v[8];
 #pragma unroll
@@ -499,7 +544,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                if (c0 + q * NT < j) fs[c0 + q * NT] = v[q];
+                if (c0 + q * NT < j) fs2[c0 + q * NT] = make_float2(v[q], v[q]);
         }
         __syncthreads();
 
@@ -511,8 +556,8 @@ __global__ void __launch_bounds__(NT, 512 / NT) rpcholesky_kernel(const SelectAr
             const int i0 = r0 + il0;
             if (!in_bounds(i0 + kGroup <= ldf, status)) continue;
             double dot[kGroup], cor[kGroup];
-            key_dots<TK>(Kt + i0, ldf, d, ks, dot);
-            correction(F + i0, ldf, j, fs, cor);
+            key_dots<TK>(Kt + i0, ldf, d, ks2, ks, dot);
+            correction(F + i0, ldf, j, fs2, cor);
             float out[kGroup];
 #pragma unroll
             for (int k = 0; k < kGroup; ++k) {
@@ -852,6 +897,199 @@ __global__ void __launch_bounds__(NT, 1) rpcholesky_resident_kernel(const Select
     cluster.sync();  // no block leaves while a peer may still write to its shared memory
 }
 
+// ---- one block per unit: keys in shared memory, factor streamed ----
+//
+// Many short units (at least one per SM, at most 2 kUnitThreads keys each) take
+// a block of kUnitThreads threads per unit, a pair of rows per thread.  The
+// block keeps the unit's transposed keys in shared memory and streams only the
+// factor columns (from L2: a wave's factors are a few tens of MB).  With one
+// block per unit no step waits on another block: the slice sum is the block's
+// own scan total, the pivot draws are taken before the first step, the pivot is
+// found by the one thread whose inclusive prefix first passes tau, and the
+// pivot's factor row is in flight while the key dots run.  Same per-row
+// arithmetic as rpcholesky_kernel.
+constexpr int kUnitThreads = 512;
+
+struct UnitSmem {
+    size_t dg, scan, uj, ks, ks2, fs2, ispiv, kt, total;
+    __host__ __device__ UnitSmem(int m, int r, int d, int tk) {
+        size_t o = 0;
+        dg = o;    o = align16(o + (size_t)m * 8);
+        scan = o;  o = align16(o + (size_t)kUnitThreads * 8);
+        uj = o;    o = align16(o + (size_t)r * 8);
+        ks = o;    o = align16(o + (size_t)d * 8);
+        ks2 = o;   o = align16(o + (size_t)d * 8);
+        fs2 = o;   o = align16(o + (size_t)r * 8);
+        ispiv = o; o = align16(o + (size_t)m);
+        kt = o;    o = align16(o + (size_t)d * m * tk);
+        total = o;
+    }
+};
+
+template <typename T, typename TK>
+__global__ void __launch_bounds__(kUnitThreads, 1) rpcholesky_unit_kernel(const SelectArgs a) {
+    constexpr int NT = kUnitThreads;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int tid = threadIdx.x;
+    const int unit = blockIdx.x;
+    const int n = a.n, d = a.d, r = a.r, m = a.m;  // m = ldf <= 2 NT
+    const int64_t ldf = a.ldf;
+    const UnitSmem L(m, r, d, (int)sizeof(TK));
+    double* dg = reinterpret_cast<double*>(smem + L.dg);
+    double* scan = reinterpret_cast<double*>(smem + L.scan);
+    double* uj = reinterpret_cast<double*>(smem + L.uj);
+    double* ks = reinterpret_cast<double*>(smem + L.ks);
+    float2* ks2 = reinterpret_cast<float2*>(smem + L.ks2);
+    float2* fs2 = reinterpret_cast<float2*>(smem + L.fs2);
+    unsigned char* ispiv = smem + L.ispiv;
+    TK* Kts = reinterpret_cast<TK*>(smem + L.kt);  // [d][m]
+    __shared__ double piv_ds;
+    __shared__ int piv_s, piv_stop;
+    __shared__ unsigned long long lmax_bits;
+
+    const T* K = static_cast<const T*>(a.K) + (size_t)unit * n * d;
+    const double* kb = a.kbar ? a.kbar + (size_t)(unit / a.bins) * d : nullptr;
+    float* F = a.F + (size_t)unit * r * ldf;
+    int* status = a.status;
+    // this thread's rows: il0 and il0 + 1 (rows >= n up to ldf are padding, F zero there)
+    const int il0 = 2 * tid;
+    const bool has = il0 < ldf;
+    const int lo = min(n, il0), hi = min(n, il0 + 2);
+
+    // ---- the pivot draws; the keys, transposed into shared memory; beta |k_i|^2
+    for (int jj = tid; jj < r; jj += NT) uj[jj] = pivot_uniform(a.seed, (uint32_t)jj, a.unit_base + (uint32_t)unit);
+    if (tid == 0) lmax_bits = 0ull;
+    __syncthreads();
+    double lmax = 0.0;
+    for (int il = il0; il < il0 + 2 && il < m; ++il) {
+        double v = 0.0;
+        if (il < n) {
+            const T* krow = K + (size_t)il * d;
+            double ss = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const T kv = krow[c];
+                double x = (double)to_f32(kv);
+                if (kb) x -= kb[c];
+                ss += x * x;
+                if constexpr (std::is_same<T, TK>::value) Kts[(size_t)c * m + il] = kb ? TK((float)x) : kv;
+                else Kts[(size_t)c * m + il] = (TK)(float)x;
+            }
+            v = a.beta * ss;
+        } else {
+            for (int c = 0; c < d; ++c) Kts[(size_t)c * m + il] = TK(0.f);
+        }
+        dg[il] = v;
+        ispiv[il] = 0;
+        lmax = fmax(lmax, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if ((tid & 31) == 0 && lmax > 0.0) atomicMax(&lmax_bits, (unsigned long long)__double_as_longlong(lmax));
+    __syncthreads();
+    const double shift = __longlong_as_double((long long)lmax_bits);
+    bool alive = isfinite(shift);
+    if (!alive && tid == 0) record_status(status, WC_ERR_NUMERIC);
+    const double hmax = 1.0;  // the shifted diagonal's maximum
+
+    double total = 0.0;
+    if (alive) {
+        double sum = 0.0;
+        for (int il = lo; il < hi; ++il) {
+            dg[il] = exp(dg[il] - shift);
+            sum += dg[il];
+        }
+        total = block_scan<NT>(sum, scan);
+    }
+
+    int final_rank = alive ? r : 0;
+    for (int j = 0; alive && j < r; ++j) {
+        // 1. the pivot: the thread whose inclusive prefix first passes
+        // t = u_j * total (else the last thread) scans its two rows
+        if (!(total > 0.0)) {
+            if (isnan(total) && tid == 0) record_status(status, WC_ERR_NUMERIC);
+            final_rank = j;
+            break;
+        }
+        const double tau = uj[j] * total;
+        const bool past = scan[tid] > tau;
+        const bool prev = tid > 0 && scan[tid - 1] > tau;
+        if ((past && !prev) || (tid == NT - 1 && !past)) {
+            double run = tid == 0 ? 0.0 : scan[tid - 1];
+            int sl = -1;
+            for (int il = lo; il < hi; ++il) {
+                run += dg[il];
+                if (run > tau) { sl = il; break; }
+            }
+            if (sl < 0) {  // rounding: last positive entry of the pair, else of the unit
+                for (int il = hi - 1; il >= lo && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                for (int il = n - 1; il >= 0 && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+            }
+            const double ds = sl >= 0 ? dg[sl] : 0.0;
+            const int stop = !(ds > a.eps * hmax);
+            if (!stop) a.piv[(size_t)unit * r + j] = sl + (unit % a.bins) * a.bin_keys;
+            piv_s = sl;
+            piv_ds = ds;
+            piv_stop = stop;
+        }
+        __syncthreads();
+        if (piv_stop) { final_rank = j; break; }
+        const int s = piv_s;
+        const double ds = piv_ds;
+        if (!in_bounds(s >= 0 && s < n, status)) {  // every thread reads the same s: all stop here
+            final_rank = j;
+            break;
+        }
+
+        // 2. the pivot key into shared memory; its factor row's loads issued
+        for (int c = tid; c < d; c += NT) {
+            const double kv = kb ? (double)to_f32(K[(size_t)s * d + c]) - kb[c] : (double)to_f32(Kts[(size_t)c * m + s]);
+            ks[c] = kv;
+            ks2[c] = make_float2((float)kv, (float)kv);
+        }
+        const float fv0 = tid < j ? ld_cg_f32(F + (int64_t)tid * ldf + s) : 0.f;
+        const float fv1 = tid + NT < j ? ld_cg_f32(F + (int64_t)(tid + NT) * ldf + s) : 0.f;
+        __syncthreads();
+
+        // 3. key dots while the factor row arrives, then the correction, the
+        // column and the downdate (the pivot's own row leaves the residual)
+        double dot[2] = {0.0, 0.0}, cor[2] = {0.0, 0.0};
+        if (has) key_dots_shared(Kts + il0, m, d, ks2, ks, dot);
+        if (tid < j) fs2[tid] = make_float2(fv0, fv0);
+        if (tid + NT < j) fs2[tid + NT] = make_float2(fv1, fv1);
+        __syncthreads();
+        if (has) {
+            correction(F + il0, ldf, j, fs2, cor);
+            const double root = sqrt(ds);
+            float out[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int il = il0 + k;
+                double f = 0.0;
+                if (il < n && !ispiv[il]) f = (exp(a.beta * dot[k] - shift) - cor[k]) / root;
+                out[k] = (float)f;
+                if (il < n) {
+                    const double nd = dg[il] - f * f;
+                    dg[il] = il == s ? 0.0 : (nd > 0.0 ? nd : 0.0);
+                    if (il == s) ispiv[il] = 1;
+                }
+            }
+            *reinterpret_cast<float2*>(F + (int64_t)j * ldf + il0) = make_float2(out[0], out[1]);
+        }
+
+        // 4. the new inclusive prefixes and total (each thread sums its own rows)
+        double sum = 0.0;
+        for (int il = lo; il < hi; ++il) sum += dg[il];
+        total = block_scan<NT>(sum, scan);
+    }
+
+    // ---- columns >= rank are zero; piv beyond rank is -1
+    if (has)
+        for (int jj = final_rank; jj < r; ++jj)
+            *reinterpret_cast<float2*>(F + (int64_t)jj * ldf + il0) = make_float2(0.f, 0.f);
+    for (int jj = final_rank + tid; jj < r; jj += NT) a.piv[(size_t)unit * r + jj] = -1;
+    if (tid == 0) a.rank[unit] = final_rank;
+}
+
 struct SelectPlan {
     int C = 0, m = 0;   // blocks per unit, rows per block
     long cap = 0;       // blocks the GPU holds at once with m rows each
@@ -1052,6 +1290,20 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     if (p.C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
 
     a.C = p.C; a.m = p.m;
+
+    // many short units: one block per unit, keys in shared memory
+    if (s.units >= nsm && s.ldf <= 2 * kUnitThreads) {
+        const size_t usmem = UnitSmem((int)s.ldf, s.r, s.d, (int)sizeof(TK)).total;
+        if (usmem + 1024 <= (size_t)max_smem) {
+            auto kern = rpcholesky_unit_kernel<T, TK>;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usmem) != cudaSuccess)
+                return WC_ERR_CUDA;
+            a.C = 1;
+            a.m = (int)s.ldf;
+            kern<<<s.units, kUnitThreads, usmem, st>>>(a);
+            return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+        }
+    }
 
     if (cudaMemsetAsync(ws + L.sync, 0, sizeof(UnitSync) * (size_t)s.units, st) != cudaSuccess) return WC_ERR_CUDA;
     return use128 ? run_select<T, TK, 128>(s, p, a, ws, st) : run_select<T, TK, 256>(s, p, a, ws, st);
