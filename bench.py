@@ -516,9 +516,10 @@ def kernel_breakdown(step):
             # modes 0, 2: the weights' partial sums; 1: attention; 3: attention over a key split
             short = "attend_gemm" if m.group(2) in ("1", "3") else "weights_gemm"
         else:
-            if "rpcholesky" in name:
-                # the streaming kernel, or the shared-memory one for few short units
-                out["select_kernel"] = "rpcholesky_resident_kernel" if "resident" in name else "rpcholesky_kernel"
+            sk = re.search(r"rpcholesky_\w*kernel", name)
+            if sk:
+                # the streaming kernel, or a shared-memory form for short units
+                out["select_kernel"] = sk.group(0)
             for key, tag in (("rpcholesky", "select"), ("gather_kernel", "gather"), ("to_half", "v_to_fp16"),
                              ("merge_c1", "merge_c1"), ("trsm_", "solve"),
                              ("weights_prep", "w_prep"), ("key_shift", "shift"),
