@@ -1090,6 +1090,270 @@ __global__ void __launch_bounds__(kUnitThreads, 1) rpcholesky_unit_kernel(const 
     if (tid == 0) a.rank[unit] = final_rank;
 }
 
+// ---- a cluster per unit, keys and factor streamed ----
+//
+// Units of 2 to kMaxCluster blocks (moderate key counts, tens of units) take the
+// streaming kernel's steps with the hand-off through distributed shared memory:
+// the blocks of a unit form a thread-block cluster; the slice sums go to every
+// block, the owner block finds the pivot and sends it, the pivot key and the
+// pivot's factor row (its own rows, so its own writes) to every block, and the
+// blocks meet at the cluster barrier.  A step then waits on no global-memory
+// flag or barrier, and each block reads and writes only its own rows of Kt and
+// F.  The pivot draws are taken before the first step; the pivots go out after
+// the last.  Same per-row arithmetic as rpcholesky_kernel.
+struct ClusterSmem {
+    size_t dg, scan, bsum, bmax, uj, ks, ks2, fs2, msg, pv, ispiv, total;
+    __host__ __device__ ClusterSmem(int m, int r, int d) {
+        size_t o = 0;
+        dg = o;    o = align16(o + (size_t)m * 8);
+        scan = o;  o = align16(o + (size_t)kThreads * 8);
+        bsum = o;  o = align16(o + (size_t)kMaxCluster * 8);
+        bmax = o;  o = align16(o + (size_t)kMaxCluster * 8);
+        uj = o;    o = align16(o + (size_t)r * 8);
+        ks = o;    o = align16(o + (size_t)d * 8);
+        ks2 = o;   o = align16(o + (size_t)d * 8);
+        fs2 = o;   o = align16(o + (size_t)r * 8);
+        msg = o;   o = align16(o + sizeof(PivMsg));
+        pv = o;    o = align16(o + (size_t)r * 4);
+        ispiv = o; o = align16(o + (size_t)m);
+        total = o;
+    }
+};
+
+template <typename T, typename TK>
+__global__ void __launch_bounds__(kThreads, 2) rpcholesky_cluster_kernel(const SelectArgs a) {
+    constexpr int NT = kThreads;
+    extern __shared__ __align__(16) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int CL = (int)cluster.num_blocks();
+    const int blk = (int)cluster.block_rank();
+    const int tid = threadIdx.x;
+    const int unit = blockIdx.x / CL;
+    const int n = a.n, d = a.d, r = a.r, m = a.m;
+    const int64_t ldf = a.ldf;
+    const int r0 = min(n, blk * m);
+    const int r1 = min(n, r0 + m);
+    const int mlen = r1 - r0;
+    // groups this block computes: its rows, and for the last block the padding
+    // up to the row stride ldf as well (F is zero there)
+    const int ng = r1 == n ? (int)((ldf - r0 + kGroup - 1) / kGroup) : (mlen + kGroup - 1) / kGroup;
+
+    const ClusterSmem L(m, r, d);
+    double* dg = reinterpret_cast<double*>(smem + L.dg);
+    double* scan = reinterpret_cast<double*>(smem + L.scan);
+    double* bsum = reinterpret_cast<double*>(smem + L.bsum);
+    double* bmax = reinterpret_cast<double*>(smem + L.bmax);
+    double* uj = reinterpret_cast<double*>(smem + L.uj);
+    double* ks = reinterpret_cast<double*>(smem + L.ks);
+    float2* ks2 = reinterpret_cast<float2*>(smem + L.ks2);
+    float2* fs2 = reinterpret_cast<float2*>(smem + L.fs2);
+    PivMsg* msg = reinterpret_cast<PivMsg*>(smem + L.msg);
+    int* pv = reinterpret_cast<int*>(smem + L.pv);
+    unsigned char* ispiv = smem + L.ispiv;
+    __shared__ int own_sl, own_stop;
+    __shared__ double own_ds;
+    __shared__ unsigned long long lmax_bits;
+
+    const T* K = static_cast<const T*>(a.K) + (size_t)unit * n * d;
+    TK* Kt = static_cast<TK*>(a.Kt) + (size_t)unit * d * ldf;
+    const double* kb = a.kbar ? a.kbar + (size_t)(unit / a.bins) * d : nullptr;
+    float* F = a.F + (size_t)unit * r * ldf;
+    int* status = a.status;
+
+    // ---- the pivot draws; the slice's keys transposed (this block's rows of
+    // the unit's copy); beta |k_i|^2
+    for (int jj = tid; jj < r; jj += NT) uj[jj] = pivot_uniform(a.seed, (uint32_t)jj, a.unit_base + (uint32_t)unit);
+    if (tid == 0) lmax_bits = 0ull;
+    __syncthreads();
+    double lmax = 0.0;
+    for (int il = tid; il < ng * kGroup; il += NT) {
+        const int i = r0 + il;
+        if (il < mlen) {
+            const T* krow = K + (size_t)i * d;
+            double ss = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const T v = krow[c];
+                double x = (double)to_f32(v);
+                if (kb) x -= kb[c];
+                ss += x * x;
+                if constexpr (std::is_same<T, TK>::value) Kt[(int64_t)c * ldf + i] = kb ? TK((float)x) : v;
+                else Kt[(int64_t)c * ldf + i] = (TK)(float)x;
+            }
+            dg[il] = a.beta * ss;
+            lmax = fmax(lmax, dg[il]);
+        } else {
+            for (int c = 0; c < d; ++c) Kt[(int64_t)c * ldf + i] = TK(0.f);
+            if (il < m) dg[il] = 0.0;
+        }
+        if (il < m) ispiv[il] = 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmax(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if ((tid & 31) == 0 && lmax > 0.0) atomicMax(&lmax_bits, (unsigned long long)__double_as_longlong(lmax));
+    __syncthreads();
+    if (tid < CL) cluster.map_shared_rank(bmax, tid)[blk] = __longlong_as_double((long long)lmax_bits);
+    cluster.sync();
+    double shift = 0.0;
+    for (int c = 0; c < CL; ++c) shift = fmax(shift, bmax[c]);
+    bool alive = isfinite(shift);
+    if (!alive && blk == 0 && tid == 0) record_status(status, WC_ERR_NUMERIC);
+    const double hmax = 1.0;  // the shifted diagonal's maximum
+
+    if (alive) {
+        for (int il = tid; il < mlen; il += NT) dg[il] = exp(dg[il] - shift);
+        __syncthreads();
+        int lo, hi;
+        chunk_of<NT>(tid, mlen, &lo, &hi);
+        double sum = 0.0;
+        for (int il = lo; il < hi; ++il) sum += dg[il];
+        const double tot = block_scan<NT>(sum, scan);
+        if (tid < CL) cluster.map_shared_rank(bsum, tid)[blk] = tot;
+        cluster.sync();
+    }
+
+    int final_rank = alive ? r : 0;
+    for (int j = 0; alive && j < r; ++j) {
+        // 1. the block whose slice holds t = u_j * sum(d), from the slice sums:
+        // every thread of every block of the unit takes the same decision
+        double total = 0.0;
+        for (int c = 0; c < CL; ++c) total += bsum[c];
+        if (!(total > 0.0)) {
+            if (isnan(total) && blk == 0 && tid == 0) record_status(status, WC_ERR_NUMERIC);
+            final_rank = j;
+            break;
+        }
+        const double tau = uj[j] * total;
+        int owner = -1;
+        double base = 0.0;
+        {
+            double run = 0.0;
+            for (int c = 0; c < CL; ++c) {
+                const double nxt = run + bsum[c];
+                if (nxt > tau) { owner = c; base = run; break; }
+                run = nxt;
+            }
+            if (owner < 0) {  // rounding left tau at the top: last block with mass
+                run = 0.0;
+                for (int c = 0; c < CL; ++c) {
+                    const double p = bsum[c];
+                    if (p > 0.0) { owner = c; base = run; }
+                    run += p;
+                }
+            }
+        }
+
+        // 2. the owner: the first thread whose inclusive prefix passes tau (else
+        // the last) scans its chunk; then the block sends the pivot, its key
+        // and its factor row (rows of this block: written by this block) to
+        // every block of the unit
+        if (blk == owner) {
+            const bool past = base + scan[tid] > tau;
+            const bool prev = tid > 0 && base + scan[tid - 1] > tau;
+            if ((past && !prev) || (tid == NT - 1 && !past)) {
+                int lo, hi;
+                chunk_of<NT>(tid, mlen, &lo, &hi);
+                double run = tid == 0 ? base : base + scan[tid - 1];
+                int sl = -1;
+                for (int il = lo; il < hi; ++il) {
+                    run += dg[il];
+                    if (run > tau) { sl = il; break; }
+                }
+                if (sl < 0) {  // rounding: last positive entry of the chunk, else of the slice
+                    for (int il = hi - 1; il >= lo && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                    for (int il = mlen - 1; il >= 0 && sl < 0; --il) if (dg[il] > 0.0) sl = il;
+                }
+                own_sl = sl;
+                own_ds = sl >= 0 ? dg[sl] : 0.0;
+                own_stop = !(own_ds > a.eps * hmax);
+            }
+            __syncthreads();
+            const int sl = own_sl;
+            if (!own_stop) {
+                const int sg = r0 + sl;
+                for (int c = tid; c < d; c += NT) {
+                    const double kv = (double)to_f32(K[(size_t)sg * d + c]) - (kb ? kb[c] : 0.0);
+                    const float2 kv2 = make_float2((float)kv, (float)kv);
+                    for (int p = 0; p < CL; ++p) {
+                        cluster.map_shared_rank(ks, p)[c] = kv;
+                        cluster.map_shared_rank(ks2, p)[c] = kv2;
+                    }
+                }
+                for (int c = tid; c < j; c += NT) {
+                    const float v = ld_cg_f32(F + (int64_t)c * ldf + sg);
+                    for (int p = 0; p < CL; ++p) cluster.map_shared_rank(fs2, p)[c] = make_float2(v, v);
+                }
+            }
+            if (tid < CL) {
+                PivMsg* mp = cluster.map_shared_rank(msg, tid);
+                mp->s = r0 + sl;
+                mp->d_s = own_ds;
+                mp->stop = own_stop;
+            }
+        }
+        cluster.sync();
+        if (msg->stop) { final_rank = j; break; }
+        const int s = msg->s;
+        const double ds = msg->d_s;
+        if (!in_bounds(s >= 0 && s < n, status)) {  // every block reads the same s: all stop here
+            final_rank = j;
+            break;
+        }
+        if (tid == 0) pv[j] = s;
+
+        // 3. column j over this block's rows, and the residual downdate (the
+        // pivot's own row leaves the residual here)
+        const double root = sqrt(ds);
+        const int spl = s - r0;
+        float* Fj = F + (int64_t)j * ldf;
+        for (int g = tid; g < ng; g += NT) {
+            const int il0 = g * kGroup;
+            const int i0 = r0 + il0;
+            if (!in_bounds(i0 + kGroup <= ldf, status)) continue;
+            double dot[kGroup], cor[kGroup] = {0.0, 0.0};
+            key_dots<TK>(Kt + i0, ldf, d, ks2, ks, dot);
+            correction(F + i0, ldf, j, fs2, cor);
+            float out[kGroup];
+#pragma unroll
+            for (int k = 0; k < kGroup; ++k) {
+                const int il = il0 + k;
+                double f = 0.0;
+                if (il < mlen && !ispiv[il]) f = (exp(a.beta * dot[k] - shift) - cor[k]) / root;
+                out[k] = (float)f;
+                if (il < mlen) {
+                    const double nd = dg[il] - f * f;
+                    dg[il] = il == spl ? 0.0 : (nd > 0.0 ? nd : 0.0);
+                    if (il == spl) ispiv[il] = 1;
+                }
+            }
+            *reinterpret_cast<float2*>(Fj + i0) = make_float2(out[0], out[1]);
+        }
+        __syncthreads();
+
+        // 4. new slice sum to every block, then close the step
+        {
+            int lo, hi;
+            chunk_of<NT>(tid, mlen, &lo, &hi);
+            double sum = 0.0;
+            for (int il = lo; il < hi; ++il) sum += dg[il];
+            const double tot = block_scan<NT>(sum, scan);
+            if (tid < CL) cluster.map_shared_rank(bsum, tid)[blk] = tot;
+        }
+        cluster.sync();
+    }
+
+    // ---- columns >= rank are zero; piv beyond rank is -1
+    for (int jj = final_rank; jj < r; ++jj) {
+        float* Fj = F + (int64_t)jj * ldf;
+        for (int g = tid; g < ng; g += NT) *reinterpret_cast<float2*>(Fj + r0 + g * kGroup) = make_float2(0.f, 0.f);
+    }
+    if (blk == 0) {
+        const int off = (unit % a.bins) * a.bin_keys;
+        for (int jj = tid; jj < r; jj += NT) a.piv[(size_t)unit * r + jj] = jj < final_rank ? pv[jj] + off : -1;
+        if (tid == 0) a.rank[unit] = final_rank;
+    }
+    cluster.sync();  // no block leaves while a peer may still write to its shared memory
+}
+
 struct SelectPlan {
     int C = 0, m = 0;   // blocks per unit, rows per block
     long cap = 0;       // blocks the GPU holds at once with m rows each
@@ -1290,6 +1554,33 @@ wc_status launch_select_t(const Shape& s, const void* K, int32_t* piv, float* F,
     if (p.C > kMaxBlocksPerUnit) return WC_ERR_UNSUPPORTED;
 
     a.C = p.C; a.m = p.m;
+
+    // units of 2 to kMaxCluster blocks: a cluster per unit
+    if (!use128 && p.C >= 2 && p.C <= kMaxCluster) {
+        auto kern = rpcholesky_cluster_kernel<T, TK>;
+        const size_t csmem = ClusterSmem(p.m, s.r, s.d).total;
+        if (csmem + 1024 <= (size_t)max_smem &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem) == cudaSuccess) {
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)p.C;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(s.units * p.C));
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = csmem;
+            cfg.stream = st;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters >= 1) {
+                a.unit0 = 0;
+                return cudaLaunchKernelEx(&cfg, kern, a) == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+            }
+        }
+        cudaGetLastError();
+    }
 
     // many short units: one block per unit, keys in shared memory
     if (s.units >= nsm && s.ldf <= 2 * kUnitThreads) {
