@@ -46,11 +46,32 @@ METRIC = "WildCat forward tokens/sec at 1 B200; select HBM GB/s and GEMM TC-util
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) of the select kernel per unit and launch on the named
-# workload: ncu's dram__bytes_read.sum + dram__bytes_write.sum on the same 8 units
-# and keys with r = 512 (669.953816 GB + 2.396056 GB against 688.268509 GB of
-# algorithmic bytes: 0.97687), applied to the algorithmic bytes at r = 2048.
+# workload, from ncu's dram__bytes_read.sum + dram__bytes_write.sum (one-pass
+# metrics) of the current select kernels:
+#   long: the same 8 units and keys with r = 512 (670.081566 GB + 2.396902 GB
+#     against 688.268509 GB of algorithmic bytes: 0.977058), applied to the
+#     algorithmic bytes at r = 2048;
+#   vit: the whole workload (149.6192 MB + 145.093376 MB over 768 units; the
+#     keys are read once and the factor stays in L2);
+#   tiny: the whole workload (193,536 bytes read, none written: the factor
+#     stays in shared memory until it is written out).
 # Other workloads: not captured.
-SELECT_DRAM_BYTES_PER_UNIT = {"long": 0.976871 * 9350143803392 / 8}
+# Each entry: (the select kernel captured, units per launch then or None where
+# the per-unit figure carries over to other unit counts, bytes per unit).
+SELECT_DRAM_CAPTURES = {
+    "long": ("rpcholesky_kernel", None, 0.977058 * 9350143803392 / 8),
+    "vit": ("rpcholesky_unit_kernel", 768, (149619200 + 145093376) / 768),
+    "tiny": ("rpcholesky_resident_kernel", 1, 193536.0),
+}
+
+
+def select_traffic(name, kernel, units, bins, center):
+    """DRAM bytes of one select launch from the capture above, or None where
+    none applies (another kernel, unit count, bins or centring)."""
+    cap = SELECT_DRAM_CAPTURES.get(name)
+    if cap is None or bins != 1 or center or cap[0] != kernel or (cap[1] is not None and cap[1] != units):
+        return None
+    return cap[2] * units
 
 
 def load_peaks():
@@ -436,8 +457,7 @@ def run_ours(args, world, rank, local):
     achieved = sb / (sel_avg * 1e-3) / 1e9
     f1, f2 = gemm_flops(w, args.bins)
     wts_avg, att_avg = sum(wts_ms) / len(wts_ms), sum(att_ms) / len(att_ms)
-    captured = w.name in SELECT_DRAM_BYTES_PER_UNIT and args.bins == 1 and not args.center
-    traffic = SELECT_DRAM_BYTES_PER_UNIT[w.name] * w.batch * w.hkv if captured else None
+    traffic = select_traffic(w.name, sel_kernel, w.batch * w.hkv, args.bins, args.center)
     tokens = job_tokens
     gather = None
     if args.gather and world > 1 and args.scaling == "strong":

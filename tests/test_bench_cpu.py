@@ -27,6 +27,21 @@ def test_algorithmic_counts_of_the_long_workload():
     assert bench.select_bytes(w, center=True) - bench.select_bytes(w) == n * r * d * 2 * w.hkv
 
 
+def test_select_traffic_applies_only_to_the_captured_kernel_and_units():
+    long_units = WORKLOADS["long"].hkv * WORKLOADS["long"].batch
+    t = bench.select_traffic("long", "rpcholesky_kernel", long_units, 1, False)
+    assert abs(t / bench.select_bytes(WORKLOADS["long"]) - 0.977058) < 1e-9
+    # the long capture carries over to other unit counts (a strong split)
+    assert bench.select_traffic("long", "rpcholesky_kernel", 1, 1, False) == t / long_units
+    # another kernel, another unit count for a whole-workload capture, bins or centring: none
+    assert bench.select_traffic("long", "rpcholesky_cluster_kernel", long_units, 1, False) is None
+    assert bench.select_traffic("vit", "rpcholesky_unit_kernel", 768, 1, False) == 149619200 + 145093376
+    assert bench.select_traffic("vit", "rpcholesky_unit_kernel", 96, 1, False) is None
+    assert bench.select_traffic("vit", "rpcholesky_unit_kernel", 768, 4, False) is None
+    assert bench.select_traffic("tiny", "rpcholesky_resident_kernel", 1, 1, True) is None
+    assert bench.select_traffic("kv", "rpcholesky_kernel", 8, 1, False) is None
+
+
 def test_reference_arm_prints_one_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
                           "--steps", "1", "--warmup", "3", "--ref-pivots", "32"],
