@@ -83,6 +83,28 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def read_stream_gbs(dev, stream, gib: int = 4, reps: int = 5) -> float:
+    """Read-only bandwidth of this GPU: the library's read probe streaming a
+    buffer far larger than L2 (outside the timed region).  The select reads
+    about five hundred bytes per byte it writes, so this figure, beside the
+    copy bandwidth of MEASURED_PEAKS.json, is the other bound on it."""
+    from coreset_attention_approximation_b200 import wildcat
+    buf = torch.empty(gib << 30, dtype=torch.uint8, device=dev)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(2):
+        wildcat.read_probe(buf, sink, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        wildcat.read_probe(buf, sink, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = buf.numel()
+    del buf
+    return nbytes / (ms * 1e-3) / 1e9
+
+
 def select_bytes(w, bins: int = 1, center: bool = False) -> float:
     """Algorithmic bytes of one select launch: per unit (per bin with bins) and
     pivot step j, one read of K (n d s_K), of the factor prefix F[:, :j] (4 n j)
@@ -452,6 +474,7 @@ def run_ours(args, world, rank, local):
     alone.pop("select_kernel", None)
 
     peaks, which = load_peaks()
+    read_gbs = read_stream_gbs(dev, stream)
     sel_avg = sum(sel_ms) / len(sel_ms)
     sb = select_bytes(w, args.bins, args.center)
     achieved = sb / (sel_avg * 1e-3) / 1e9
@@ -488,6 +511,8 @@ def run_ours(args, world, rank, local):
             "bound": "hbm", "kernel": sel_kernel + " (select)", "achieved": achieved,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
             "traffic": traffic, "peak_source": which,
+            # the read-only stream this GPU reaches (the library's read probe), beside the copy peak
+            "peak_read_gbs": read_gbs, "frac_read": achieved / read_gbs,
             "algorithmic_bytes_per_launch": sb, "launch_ms": sel_avg,
         },
         "stages_ms": {"select": sel_avg, "weights": wts_avg, "attend": att_avg},

@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwildcat.so")
 OBJDIR = os.path.join(HERE, "_build")
 SOURCES = ["api.cu", "select.cu", "weights.cu", "expmm_simt.cu", "expmm_tc.cu", "attend.cu", "noalloc.cu",
-           "center.cu"]
+           "center.cu", "stream_probe.cu"]
 HEADERS = ["wc_common.cuh", "wc_internal.h", "wc_expmm.cuh", "wc_tc.cuh", "wc_exp2.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

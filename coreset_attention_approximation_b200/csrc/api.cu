@@ -246,6 +246,12 @@ wc_status wc_selftest_exp2(const float* x, float* y, int64_t n, int32_t method, 
     return launch_exp2_selftest(x, y, n, method, static_cast<cudaStream_t>(stream));
 }
 
+wc_status wc_read_bandwidth_probe(const void* buf, int64_t bytes, uint32_t* sink, void* stream) {
+    if (!buf || !sink || bytes <= 0 || (bytes & 15) || ((uintptr_t)buf & 15u) || ((uintptr_t)sink & 3u))
+        return WC_ERR_INVALID;
+    return launch_read_probe(buf, bytes, sink, static_cast<cudaStream_t>(stream));
+}
+
 const char* wc_status_string(wc_status status) {
     switch (status) {
         case WC_OK: return "ok";

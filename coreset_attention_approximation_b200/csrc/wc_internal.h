@@ -100,6 +100,7 @@ Shape bin_view(const Shape& s);
 WsLayout make_layout(const Shape& s);
 
 // Kernel launchers (each returns WC_OK or WC_ERR_CUDA / WC_ERR_UNSUPPORTED).
+wc_status launch_read_probe(const void* buf, int64_t bytes, uint32_t* sink, cudaStream_t st);
 wc_status launch_select(const Shape& s, const void* K, int32_t* piv, float* F, int32_t* rank,
                         char* ws, cudaStream_t st);
 wc_status launch_gather(const Shape& s, const void* K, const int32_t* piv, const float* F,

@@ -44,7 +44,7 @@ class WcShape(ctypes.Structure):
 EXPORTS = [
     "wc_f_ld", "wc_workspace_bytes", "wc_forward_workspace_bytes", "wc_select", "wc_weights", "wc_attend",
     "wc_forward", "wc_check_device_status", "wc_selftest_wait_timeout", "wc_status_string",
-    "wc_attend_noalloc", "wc_selftest_exp2",
+    "wc_attend_noalloc", "wc_selftest_exp2", "wc_read_bandwidth_probe",
 ]
 
 _lib = None
@@ -86,6 +86,8 @@ def lib():
         L.wc_attend_noalloc.argtypes, L.wc_attend_noalloc.restype = [sp, vp, vp, vp, vp, vp, vp], i32
         L.wc_selftest_exp2.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int32, vp]
         L.wc_selftest_exp2.restype = i32
+        L.wc_read_bandwidth_probe.argtypes = [vp, ctypes.c_int64, vp, vp]
+        L.wc_read_bandwidth_probe.restype = i32
         _lib = L
     return _lib
 
@@ -337,6 +339,14 @@ def check_device_status(ws, stream=None) -> int:
 
 def selftest_wait_timeout(ws, timeout_ms, stream=None) -> int:
     return int(lib().wc_selftest_wait_timeout(_ptr(ws), ws.numel(), timeout_ms, _stream(stream)))
+
+
+def read_probe(buf, sink, stream=None):
+    """Reads the CUDA tensor `buf` once as a read-only stream (the read
+    bandwidth probe); `sink` (one int32 on the device) receives the XOR of its
+    32-bit words."""
+    _check(lib().wc_read_bandwidth_probe(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), _stream(stream)),
+           "wc_read_bandwidth_probe")
 
 
 def selftest_exp2(x, method=0, stream=None):

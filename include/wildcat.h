@@ -210,12 +210,23 @@ wc_status wc_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_m
  *             2^n added to the exponent; relative error <= 2^-13.5 for
  *             -125 <= x <= 127, about 2^-125 returned below -125
  *   method 1  the exponential unit (ex2.approx.ftz.f32)
- * The kernels run part of every row's exponentials with method 0 to relieve
- * the exponential unit, which the tensor pipe otherwise waits for.  For
- * tests; asynchronous on `stream`; WC_ERR_INVALID for n < 0, a null or
- * misaligned pointer or another method.
+ * The kernels can run part of every row's exponentials with method 0 to
+ * relieve the exponential unit (a build option, off by default: on the
+ * measured workloads it was no faster).  For tests; asynchronous on `stream`;
+ * WC_ERR_INVALID for n < 0, a null or misaligned pointer or another method.
  */
 wc_status wc_selftest_exp2(const float* x, float* y, int64_t n, int32_t method, void* stream);
+
+/*
+ * Reads buf[0 .. bytes) (device memory, 16-byte aligned, bytes a positive
+ * multiple of 16) once as a plain read-only stream and writes the XOR of its
+ * 32-bit words to *sink (device memory, 4-byte aligned).  A measurement aid,
+ * no step of the method: the read bandwidth it reaches (bytes / its time) is
+ * the denominator to set beside the copy bandwidth for a kernel that, like
+ * the select, reads far more than it writes.  Asynchronous on `stream`;
+ * WC_ERR_INVALID for a null or misaligned pointer or a bad size.
+ */
+wc_status wc_read_bandwidth_probe(const void* buf, int64_t bytes, uint32_t* sink, void* stream);
 
 /*
  * attend_noalloc — the same result as wc_attend, for callers that cannot
