@@ -31,10 +31,18 @@
 // cooperatively (all blocks co-resident); every wait gives up after the
 // shape's timeout and records WC_ERR_TIMEOUT.
 //
-// Few short units (all of them on the GPU at once, each unit's keys and factor
-// within the shared memory of a cluster of up to 8 blocks) take the resident
-// variant below instead: the same steps on shared-memory copies, the blocks
-// meeting at the cluster barrier.
+// Three forms of the same steps serve shorter units (launch_select_t picks,
+// in this order):
+//   * resident: few units, each one's keys and factor within the shared
+//     memory of a cluster of up to 8 blocks, all units on the GPU at once;
+//     nothing streams, the blocks meet at the cluster barrier;
+//   * cluster: units of 2 to 8 blocks; the blocks of a unit form a cluster
+//     and hand the step over through distributed shared memory instead of
+//     global-memory flags and barriers; keys and factor stream as above;
+//   * unit: many units (at least one per SM) of at most 1024 keys; one block
+//     per unit keeps the unit's keys in shared memory and streams the factor.
+// All forms do every row's arithmetic in the same order as the streaming
+// kernel, so the factor agrees with it wherever the slice boundaries do.
 #include <cooperative_groups.h>
 #include <type_traits>
 
