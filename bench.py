@@ -54,7 +54,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 #   vit: the whole workload (149.6192 MB + 145.093376 MB over 768 units; the
 #     keys are read once and the factor stays in L2);
 #   tiny: the whole workload (193,536 bytes read, none written: the factor
-#     stays in shared memory until it is written out).
+#     stays in shared memory until it is written out);
+#   diffusion: the whole workload (9.135514 GB + 109.580544 MB over 32 units:
+#     keys and much of the factor stay in L2).
 # Other workloads: not captured.
 # Each entry: (the select kernel captured, units per launch then or None where
 # the per-unit figure carries over to other unit counts, bytes per unit).
@@ -62,6 +64,7 @@ SELECT_DRAM_CAPTURES = {
     "long": ("rpcholesky_kernel", None, 0.977058 * 9350143803392 / 8),
     "vit": ("rpcholesky_unit_kernel", 768, (149619200 + 145093376) / 768),
     "tiny": ("rpcholesky_resident_kernel", 1, 193536.0),
+    "diffusion": ("rpcholesky_cluster_kernel", 32, (9135514000 + 109580544) / 32),
 }
 
 

@@ -40,6 +40,8 @@ def test_select_traffic_applies_only_to_the_captured_kernel_and_units():
     assert bench.select_traffic("vit", "rpcholesky_unit_kernel", 768, 4, False) is None
     assert bench.select_traffic("tiny", "rpcholesky_resident_kernel", 1, 1, True) is None
     assert bench.select_traffic("kv", "rpcholesky_kernel", 8, 1, False) is None
+    assert bench.select_traffic("diffusion", "rpcholesky_kernel", 32, 1, False) is None
+    assert bench.select_traffic("diffusion", "rpcholesky_cluster_kernel", 32, 1, False) == 9135514000 + 109580544
 
 
 def test_reference_arm_prints_one_json_line():
