@@ -34,6 +34,11 @@ def test_debug_build_matches_the_oracle(debug_lib):
     compare(*make_inputs(w), w.r, seed=0, tol_w=1e-5)
     w = WORKLOADS["kv"].replace(hq=8, hkv=2, n_k=4096, n_q=256, r=256)
     compare_next(*make_inputs(w, seed=32), w.r, seed=32, bins=4, center=True, tol_w=2e-3)
+    # the select's forms for shorter units: one block per unit, a cluster per unit
+    w = WORKLOADS["vit"].replace(batch=2, hq=80, hkv=80, n_q=128)
+    compare(*make_inputs(w, seed=34), w.r, seed=34, tol_w=2e-3)
+    w = WORKLOADS["diffusion"].replace(r=48, n_q=256)
+    compare(*make_inputs(w, seed=35), w.r, seed=35, tol_w=2e-3)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
