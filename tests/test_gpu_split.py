@@ -67,3 +67,38 @@ def test_unit_base_changes_the_draws():
     a = _run(Q, K, V, W.r)["piv"].numpy()
     b = _run(Q, K, V, W.r, unit_base=5)["piv"].numpy()
     assert not np.array_equal(a, b)
+
+
+def _select_kernels(K, r, **kw):
+    import re
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        wildcat.select(K.cuda(), r, seed=3, **kw)
+        torch.cuda.synchronize()
+    return {m.group(0) for e in prof.events() if e.device_type.name == "CUDA"
+            for m in [re.search(r"rpcholesky_\w*kernel", e.name)] if m}
+
+
+def test_strong_split_across_select_forms():
+    # 160 short heads: one block per unit in one call; 80 per part, fewer than
+    # the SMs, take a cluster per unit.  The pivots do not depend on the form;
+    # the outputs agree to the bf16 path's tolerance, since the attention and
+    # weights GEMMs also split their work by the head count (fp16 P rounded
+    # against other running maxima, partial sums merged in another order).
+    w = WORKLOADS["vit"].replace(batch=2, hq=80, hkv=80, n_q=64)
+    U, group = w.batch * w.hkv, w.hq // w.hkv
+    Q, K, V, _, _, _ = bench.local_problem(w, 3, 1, 0, "strong")
+    full = _run(Q, K, V, w.r)
+    kinds = {frozenset(_select_kernels(K, w.r))}
+    piv = full["piv"].reshape(U, w.r)
+    out = full["out"].reshape(U, group, w.n_q, w.dv)
+    for k in range(2):
+        Qk, Kk, Vk, wl, base, _ = bench.local_problem(w, 3, 2, k, "strong")
+        kinds.add(frozenset(_select_kernels(Kk, w.r, unit_base=base)))
+        part = _run(Qk, Kk, Vk, w.r, unit_base=base)
+        n = wl.batch
+        assert torch.equal(part["piv"].reshape(n, w.r), piv[base:base + n])
+        got = part["out"].reshape(n, group, w.n_q, w.dv)
+        for u in range(n):
+            assert rel_err(got[u].numpy(), out[base + u].numpy()) <= 2e-3
+    assert kinds == {frozenset({"rpcholesky_unit_kernel"}), frozenset({"rpcholesky_cluster_kernel"})}
